@@ -1,0 +1,269 @@
+/*
+ * msa.h -- C ABI of libmsa.so, the B200 (sm_100a) hot path of Memory Sparse
+ * Attention (MSA).
+ *
+ * The method (MSA: "Memory Sparse Attention for Efficient End-to-End Memory
+ * Model Scaling to 100M Tokens"):
+ *   - offline memory encoding: documents are cut into fixed-length chunks and
+ *     each chunk's K, V and router key K_r are mean-pooled; keys carry
+ *     document-wise RoPE (positions restart at 0 in each document)
+ *     [Evermind summary sec. 2; b-lab.team summary item 1 and pipeline stage
+ *     "Global Memory Encoding"];
+ *   - online routing: cosine similarity between the query's router projection
+ *     Q_r and every pooled router key, averaged over router heads, maxed over
+ *     query tokens and over a document's chunks, then the top-k documents
+ *     [b-lab.team item 1, Scalable Sparse Attention; pipeline stage "Online
+ *     Routing & Context Assembly"];
+ *   - sparse generation: the selected documents' pooled K/V are placed ahead
+ *     of the query's local K/V, the query's positions start at k (Global RoPE),
+ *     and attention runs over that context [b-lab.team item 1, Global RoPE;
+ *     pipeline stage "Sparse Generation"].
+ *
+ * Conventions for every call:
+ *   - Memory: the CALLER owns every buffer it passes (device memory, or pinned
+ *     host memory where stated).  The library never frees caller memory and
+ *     allocates device memory only inside msa_memory_create (small index and
+ *     RoPE tables, freed by msa_memory_destroy).  Scratch space for a call is
+ *     passed in as `workspace`; its size comes from the matching *_workspace_size
+ *     query.  Device pointers must be 16-byte aligned.
+ *   - Layouts are dense row-major; "token-major" means [token][head][dim].
+ *     Element type is the memory's dtype (fp32 or bf16) unless stated;
+ *     scores and running states are fp32, ids int32.
+ *   - Asynchrony: arguments are validated on the host before anything is
+ *     enqueued; work is then enqueued on `stream` and the call returns.  A
+ *     rejected call enqueues nothing.
+ *   - Errors: every call returns an msa_status; nothing aborts or throws.
+ *     msa_last_error() gives a thread-local message for the last failure.
+ *     Conditions that only the device can see (an id >= n_docs, a local cache
+ *     that would overflow, a bounded wait that ran out) are recorded in a
+ *     device error word and skipped; msa_device_error() reads and clears it.
+ *   - Threads: a msa_memory handle is immutable after creation and may be
+ *     used from several threads; calls that share output buffers must be
+ *     ordered by the caller.
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st *msa_stream;
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1,   /* a bad argument; nothing was enqueued */
+  MSA_ERR_UNSUPPORTED = 2,   /* a shape this build has no kernel for */
+  MSA_ERR_CUDA = 3,          /* a CUDA runtime error (launch or copy) */
+  MSA_ERR_OUT_OF_MEMORY = 4, /* msa_memory_create could not allocate its tables */
+  MSA_ERR_TIMEOUT = 5,       /* a bounded device wait ran out (device error word) */
+  MSA_ERR_STATE = 6,         /* a device-side bounds check fired (device error word) */
+} msa_status;
+
+typedef enum { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype;
+
+/* Device error word bits reported by msa_device_error(). */
+#define MSA_DEVERR_BAD_DOC_ID 0x1u      /* an id outside [0, n_docs) reached attention */
+#define MSA_DEVERR_CACHE_OVERFLOW 0x2u  /* cache_len + tokens > cache_capacity */
+#define MSA_DEVERR_WAIT_TIMEOUT 0x4u    /* a pipeline barrier wait ran out */
+
+/*
+ * The memory's shape.  Documents [Evermind sec. 2: the corpus is split into
+ * documents, each cut into fixed-length chunks]:
+ *   doc_token_offsets : HOST array [n_docs + 1], offsets[0] = 0, strictly
+ *                       increasing (no empty document); copied at create.
+ *   chunk_len         : tokens per chunk (2..64); the last chunk of a document
+ *                       may be shorter and is averaged over its own length.
+ * Content K/V: n_kv_heads x head_dim (head_dim 64 or 128).  Router keys:
+ * n_router_heads x router_dim (router_dim 16..128, a power of two;
+ * n_router_heads * router_dim a multiple of 64 for bf16).
+ * rope_theta: RoPE base (NeoX rotate-half); the pages give none, 1e6 is the
+ * Qwen3 value.  max_local_position: local (query/decode) RoPE positions must
+ * stay below this; document positions are covered automatically.
+ */
+typedef struct {
+  int32_t n_docs;
+  const int64_t *doc_token_offsets;
+  int32_t chunk_len;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t n_router_heads;
+  int32_t router_dim;
+  msa_dtype dtype;
+  double rope_theta;
+  int32_t max_local_position;
+} msa_memory_config;
+
+typedef struct msa_memory msa_memory;
+
+typedef struct {
+  int64_t n_tokens;
+  int64_t n_chunks;          /* total chunks C */
+  int32_t max_doc_chunks;    /* chunks of the longest document */
+  int64_t max_doc_tokens;
+  size_t elem_bytes;         /* 4 (fp32) or 2 (bf16) */
+  size_t router_key_bytes;   /* router store [C][H_r][d_r] */
+  size_t content_bytes;      /* content store [C][2][H_kv][D]: K then V per chunk */
+  size_t doc_content_stride; /* bytes of one document's content at max_doc_chunks */
+} msa_memory_info;
+
+/* Build the memory description and its device tables (chunk->document map,
+ * document offsets, fp32 RoPE cos/sin table computed in fp64) on the current
+ * CUDA device.  Errors: INVALID_ARG (bad config), UNSUPPORTED (shape without a
+ * kernel), OUT_OF_MEMORY, CUDA. */
+MSA_API msa_status msa_memory_create(const msa_memory_config *cfg, msa_memory **out);
+MSA_API msa_status msa_memory_destroy(msa_memory *mem);
+MSA_API msa_status msa_memory_get_info(const msa_memory *mem, msa_memory_info *out);
+/* First chunk of every document, written to the HOST array out[n_docs + 1]. */
+MSA_API msa_status msa_memory_doc_chunk_offsets(const msa_memory *mem, int64_t *out);
+
+/*
+ * Offline encoding of documents [doc_begin, doc_begin + doc_count)
+ * [b-lab.team pipeline stage "Global Memory Encoding"; Evermind sec. 2 chunk
+ * mean pooling; b-lab.team item 1 Document-wise RoPE].
+ *   K, V   : device, token-major [n][n_kv_heads][head_dim], K before RoPE
+ *   Kr     : device, token-major [n][n_router_heads][router_dim]
+ *            where n = tokens of those documents; row 0 is the first token of
+ *            document doc_begin.
+ * Writes, for every chunk c of those documents:
+ *   content[c][0] = mean over the chunk of RoPE(K_t, t - doc_start)
+ *   content[c][1] = mean of V_t
+ *   router_keys[c][h] = mean of Kr_t over the chunk, divided by
+ *                       max(|mean|, 1e-12) per router head: the pooled router
+ *                       key stored with unit norm, so routing needs no norms
+ *   router_mean[c][h] (optional, may be NULL) = the un-normalised mean.
+ * content may be device memory or pinned host memory (written in place over
+ * the host link).  Sums are fp32 pairwise trees; stores round to nearest even.
+ */
+MSA_API msa_status msa_encode_memory(const msa_memory *mem, int32_t doc_begin,
+                             int32_t doc_count, const void *K, const void *V,
+                             const void *Kr, void *router_keys, void *content,
+                             void *router_mean, msa_stream stream);
+
+/* Fill a running routing state (fp32, `count` entries) with -inf. */
+MSA_API msa_status msa_route_reset(float *state, int64_t count, msa_stream stream);
+
+/* Scratch bytes msa_route needs for this batch / tokens / k. */
+MSA_API size_t msa_route_workspace_size(const msa_memory *mem, int32_t batch,
+                                int32_t tokens, int32_t k);
+
+/*
+ * Online routing [b-lab.team item 1 and stage "Online Routing & Context
+ * Assembly"]:
+ *   s[b,t,c]   = (1/H_r) sum_h <Qr[b,t,h], Kr_c,h> / (|Qr[b,t,h]| |Kr_c,h|)
+ *   state[b,d] = max(state[b,d], max_{t < tokens, c in chunks(d)} s[b,t,c])
+ *   ids[b,:]   = the k documents with the largest state[b,.] by (score
+ *                descending, id ascending), excluding documents whose
+ *                exclude[b,d] != 0; scores[b,:] their states.
+ *   router_keys : device [C][H_r][d_r] as written by msa_encode_memory
+ *   Qr          : device [batch][tokens][H_r][d_r]; tokens may be 0 (top-k
+ *                 of the state only)
+ *   state       : device [batch][n_docs] fp32, read and updated (the running
+ *                 max over every token routed so far; reset with -inf)
+ *   exclude     : device [batch][n_docs] uint8 or NULL
+ *   ids, scores : device [batch][k]; k in [1, min(n_docs, 64)]
+ * Errors: INVALID_ARG (k out of range, fewer eligible documents than k is NOT
+ * checked: excluded documents then fill the tail with -inf scores), CUDA.
+ */
+MSA_API msa_status msa_route(const msa_memory *mem, const void *router_keys,
+                     const void *Qr, int32_t batch, int32_t tokens, int32_t k,
+                     const uint8_t *exclude, float *state, int32_t *ids,
+                     float *scores, void *workspace, size_t workspace_bytes,
+                     msa_stream stream);
+
+/* Scratch bytes msa_sparse_attend needs. */
+MSA_API size_t msa_attend_workspace_size(const msa_memory *mem, int32_t batch,
+                                 int32_t tokens, int32_t k, int32_t n_q_heads);
+
+/*
+ * Sparse generation [b-lab.team item 1 Scalable Sparse Attention and Global
+ * RoPE; stage "Sparse Generation"].  For query b, its `tokens` new tokens are
+ * appended to the local cache and attend over
+ *   [pooled K/V of every chunk of ids[b,0..k-1], in rank order, all visible]
+ *   ++ [local cache rows 0..j] (causal: new token i sits at local index
+ *      j = cache_len[b] + i)
+ * with Q and the new K rotated at position pos_offset + j (pos_offset = k is
+ * the pages' Global RoPE), softmax scale 1/sqrt(head_dim), and query head h
+ * reading kv head h / (n_q_heads / n_kv_heads).
+ *   content        : device [C][2][H_kv][D] (msa_encode_memory's store)
+ *   ids            : device [batch][k] int32
+ *   Q              : device [batch][tokens][n_q_heads][D], before RoPE
+ *   K_new, V_new   : device [batch][tokens][H_kv][D], K before RoPE
+ *   K_cache, V_cache : device [batch][cache_capacity][H_kv][D]; rows below
+ *                    cache_len[b] are read (K already rotated), the new rows
+ *                    are written
+ *   cache_len      : device [batch] int32, advanced by `tokens` when the work
+ *                    completes (stream order)
+ *   O              : device [batch][tokens][n_q_heads][D]
+ * Requires pos_offset >= 0 and pos_offset + cache_capacity <=
+ * max_local_position; n_q_heads a multiple of n_kv_heads with a group of at
+ * most 16.  A cache that would overflow or an id out of range is skipped and
+ * flagged in the device error word.
+ */
+MSA_API msa_status msa_sparse_attend(const msa_memory *mem, const void *content,
+                             const int32_t *ids, int32_t batch, int32_t k,
+                             int32_t tokens, int32_t n_q_heads, const void *Q,
+                             const void *K_new, const void *V_new,
+                             void *K_cache, void *V_cache, int32_t *cache_len,
+                             int32_t cache_capacity, int32_t pos_offset,
+                             void *O, void *workspace, size_t workspace_bytes,
+                             msa_stream stream);
+
+/* Per-layer decode state, every buffer owned by the caller (see msa_step). */
+typedef struct {
+  int32_t batch;
+  int32_t top_k;
+  int32_t n_q_heads;
+  int32_t cache_capacity;
+  int32_t pos_offset;        /* Global RoPE offset, normally top_k */
+  float *state;              /* device [batch][n_docs] running max */
+  int32_t *ids;              /* device [batch][top_k] */
+  float *scores;             /* device [batch][top_k] */
+  void *k_cache;             /* device [batch][cache_capacity][H_kv][D] */
+  void *v_cache;
+  int32_t *cache_len;        /* device [batch] */
+  void *workspace;
+  size_t workspace_bytes;    /* >= msa_step_workspace_size(...) */
+} msa_decode_state;
+
+MSA_API size_t msa_step_workspace_size(const msa_memory *mem, int32_t batch, int32_t k,
+                               int32_t n_q_heads);
+
+/*
+ * One routed decode step of one layer for every query of the batch
+ * [b-lab.team stages "Online Routing & Context Assembly" and "Sparse
+ * Generation", run per generated token]: route the new token with the running
+ * state (so the result equals routing over every token so far), take the
+ * top-k, then attend with the new token appended to the local cache.
+ *   Qr_tok : device [batch][H_r][d_r];  Q_tok : [batch][n_q_heads][D]
+ *   K_tok, V_tok : [batch][H_kv][D];     O_tok : [batch][n_q_heads][D]
+ */
+MSA_API msa_status msa_step(const msa_memory *mem, const void *router_keys,
+                    const void *content, const msa_decode_state *st,
+                    const void *Qr_tok, const void *Q_tok, const void *K_tok,
+                    const void *V_tok, void *O_tok, msa_stream stream);
+
+/* Read and clear the device error word of the current device (synchronises
+ * `stream`).  *bits receives the MSA_DEVERR_* bits; returns MSA_ERR_TIMEOUT or
+ * MSA_ERR_STATE when a bit was set, else MSA_OK. */
+MSA_API msa_status msa_device_error(uint32_t *bits, msa_stream stream);
+
+MSA_API const char *msa_status_string(msa_status s);
+MSA_API const char *msa_last_error(void);
+/* Library version as major*10000 + minor*100 + patch. */
+MSA_API int32_t msa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MSA_H_ */

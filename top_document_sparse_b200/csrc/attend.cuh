@@ -1,0 +1,480 @@
+// attend.cuh -- sparse generation (MSA, b-lab.team summary item 1 "Scalable
+// Sparse Attention" and "Global RoPE", stage "Sparse Generation"):
+// the new tokens attend over [pooled K/V of the retrieved documents' chunks,
+// rank order, all visible] ++ [local cache rows 0..j, causal], with Q and the
+// new K rotated at pos_offset + j.
+//
+// Kernels:
+//   append_kernel         rotate the new K rows, write K/V into the local cache
+//   attend_simt_kernel    fp32 path (CUDA cores, one warp per query head)
+//   attend_mma_kernel     bf16 path: per (query, kv head, token, context
+//                         split) CTA, 4 warps stream 16-row context blocks
+//                         (cp.async, double-buffered, XOR-swizzled smem) and
+//                         run S = Q K^T and O += P V on mma.sync with an
+//                         online softmax; the GQA group's heads are the M rows
+//   attend_combine_kernel merge context splits (log-sum-exp) and advance
+//                         cache_len
+#pragma once
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace msa {
+
+constexpr int kMaxMemRows = 4096;  // retrieved chunks per query (k * chunks per doc)
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Chunk list of query b's retrieved documents in rank order -> table[0..n_mem).
+// Ids outside [0, n_docs) contribute no rows and raise MSA_DEVERR_BAD_DOC_ID.
+// slot_of_rank (nullable, [B][k]): chunk rows of rank r start at
+// slot_of_rank[b][r] * slot_chunks instead of doc_chunk_off[id].
+__device__ __forceinline__ int build_chunk_table(const int32_t *__restrict__ ids_b, int k,
+                                                 const int64_t *__restrict__ doc_chunk_off,
+                                                 int n_docs, const int32_t *__restrict__ slots_b,
+                                                 int slot_chunks, int *table, int *pre,
+                                                 int table_cap) {
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int r = 0; r < k; ++r) {
+      pre[r] = acc;
+      const int d = ids_b[r];
+      int cnt = 0;
+      if (d >= 0 && d < n_docs) {
+        cnt = static_cast<int>(doc_chunk_off[d + 1] - doc_chunk_off[d]);
+      } else {
+        raise_device_error(MSA_DEVERR_BAD_DOC_ID);
+      }
+      if (acc + cnt > table_cap) cnt = 0;  // host validation keeps this unreachable
+      acc += cnt;
+    }
+    pre[k] = acc;
+  }
+  __syncthreads();
+  for (int r = 0; r < k; ++r) {
+    const int cnt = pre[r + 1] - pre[r];
+    if (cnt == 0) continue;
+    const int d = ids_b[r];
+    const int64_t base = slots_b ? static_cast<int64_t>(slots_b[r]) * slot_chunks : doc_chunk_off[d];
+    for (int jj = threadIdx.x; jj < cnt; jj += blockDim.x) table[pre[r] + jj] = static_cast<int>(base + jj);
+  }
+  __syncthreads();
+  return pre[k];
+}
+
+// ---------------------------------------------------------------- append
+// grid (B * T); thread i handles head h = i / (D/8) and the rotate-half pairs
+// [4q, 4q+4) of that head (K) plus 8 elements of V.
+template <typename T>
+__global__ void append_kernel(const T *__restrict__ K_new, const T *__restrict__ V_new, int T_tok,
+                              int H_kv, int D, T *__restrict__ K_cache, T *__restrict__ V_cache,
+                              const int32_t *__restrict__ cache_len, int cap, int pos_offset,
+                              const float2 *__restrict__ rope) {
+  const int b = blockIdx.x / T_tok, i = blockIdx.x % T_tok;
+  const int j = cache_len[b] + i;
+  if (j >= cap || j < 0) {
+    if (threadIdx.x == 0) raise_device_error(MSA_DEVERR_CACHE_OVERFLOW);
+    return;
+  }
+  const int per_head = D / 8;
+  const int h = threadIdx.x / per_head;
+  if (h >= H_kv) return;
+  const int i0 = (threadIdx.x % per_head) * 4;
+  const int half = D / 2;
+  const int64_t src = (static_cast<int64_t>(b) * T_tok + i) * H_kv * D + h * D;
+  const int64_t dst = (static_cast<int64_t>(b) * cap + j) * H_kv * D + h * D;
+  float a[4], c[4], lo[4], hi[4];
+  load4(K_new + src + i0, a);
+  load4(K_new + src + half + i0, c);
+  const float2 *cs = rope + static_cast<int64_t>(pos_offset + j) * half + i0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 r = cs[e];
+    lo[e] = a[e] * r.x - c[e] * r.y;
+    hi[e] = c[e] * r.x + a[e] * r.y;
+  }
+  store4(K_cache + dst + i0, lo);
+  store4(K_cache + dst + half + i0, hi);
+  float v[4];
+  load4(V_new + src + i0, v);
+  store4(V_cache + dst + i0, v);
+  load4(V_new + src + half + i0, v);
+  store4(V_cache + dst + half + i0, v);
+}
+
+// ---------------------------------------------------------------- fp32 path
+// grid (B * T), block H_q * 32: warp h owns query head h; lane owns the
+// elements lane + 32u of the head (a rotate-half partner lives in the same
+// lane because D/2 is a multiple of 32).
+template <typename T, int D>
+__global__ void __launch_bounds__(512)
+attend_simt_kernel(const T *__restrict__ content, const int32_t *__restrict__ ids, int k,
+                   const int64_t *__restrict__ doc_chunk_off, int n_docs,
+                   const int32_t *__restrict__ slots, int slot_chunks, int H_kv, int H_q,
+                   const T *__restrict__ Q, int T_tok, const T *__restrict__ K_cache,
+                   const T *__restrict__ V_cache, const int32_t *__restrict__ cache_len, int cap,
+                   int pos_offset, const float2 *__restrict__ rope, float scale,
+                   T *__restrict__ O) {
+  constexpr int U = D / 32;
+  __shared__ int table[kMaxMemRows];
+  __shared__ int pre[kMaxTopK + 1];
+  const int b = blockIdx.x / T_tok, i = blockIdx.x % T_tok;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_mem = build_chunk_table(ids + static_cast<int64_t>(b) * k, k, doc_chunk_off, n_docs,
+                                      slots ? slots + static_cast<int64_t>(b) * k : nullptr,
+                                      slot_chunks, table, pre, kMaxMemRows);
+  const int j = cache_len[b] + i;
+  const int h = warp;
+  if (h >= H_q) return;
+  T *out = O + ((static_cast<int64_t>(b) * T_tok + i) * H_q + h) * D;
+  if (j >= cap) {  // the append kernel has flagged the overflow
+    for (int u = 0; u < U; ++u) out[lane + 32 * u] = Elem<T>::from_f(0.0f);
+    return;
+  }
+  const int g = h / (H_q / H_kv);
+  const int half = D / 2;
+  float q[U];
+  {
+    const T *qs = Q + ((static_cast<int64_t>(b) * T_tok + i) * H_q + h) * D;
+    float x[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) x[u] = Elem<T>::to_f(qs[lane + 32 * u]);
+    const float2 *cs = rope + static_cast<int64_t>(pos_offset + j) * half;
+#pragma unroll
+    for (int u = 0; u < U / 2; ++u) {
+      const float2 r = cs[lane + 32 * u];
+      q[u] = x[u] * r.x - x[u + U / 2] * r.y;
+      q[u + U / 2] = x[u + U / 2] * r.x + x[u] * r.y;
+    }
+  }
+  float m = -INFINITY, l = 0.0f, acc[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) acc[u] = 0.0f;
+  const int n_ctx = n_mem + j + 1;
+  const int64_t kv = static_cast<int64_t>(H_kv) * D;
+  for (int x = 0; x < n_ctx; ++x) {
+    const T *kr, *vr;
+    if (x < n_mem) {
+      kr = content + static_cast<int64_t>(table[x]) * 2 * kv + g * D;
+      vr = kr + kv;
+    } else {
+      const int64_t row = (static_cast<int64_t>(b) * cap + (x - n_mem)) * kv + g * D;
+      kr = K_cache + row;
+      vr = V_cache + row;
+    }
+    float dot = 0.0f;
+#pragma unroll
+    for (int u = 0; u < U; ++u) dot = fmaf(q[u], Elem<T>::to_f(kr[lane + 32 * u]), dot);
+    dot = warp_sum(dot) * scale;
+    const float m_new = fmaxf(m, dot);
+    const float alpha = expf(m - m_new);
+    const float p = expf(dot - m_new);
+    l = l * alpha + p;
+#pragma unroll
+    for (int u = 0; u < U; ++u) acc[u] = fmaf(p, Elem<T>::to_f(vr[lane + 32 * u]), acc[u] * alpha);
+    m = m_new;
+  }
+  const float inv = 1.0f / l;
+#pragma unroll
+  for (int u = 0; u < U; ++u) out[lane + 32 * u] = Elem<T>::from_f(acc[u] * inv);
+}
+
+// ---------------------------------------------------------------- bf16 path
+constexpr int kAttWarps = 4;
+constexpr int kAttRows = 16;  // context rows per warp block
+
+template <int D>
+struct AttSmem {
+  static constexpr int kBlockBytes = kAttRows * D * 2;       // one K or V block
+  static constexpr int kWarpBytes = 2 /*stages*/ * 2 /*K,V*/ * kBlockBytes;
+  static constexpr int kQBytes = 16 * D * 2;
+  static constexpr int kMergeBytes = kAttWarps * 16 * (D + 2) * 4;
+  static constexpr int kRing = kAttWarps * kWarpBytes;
+  static constexpr int kFixed =
+      (kRing > kMergeBytes ? kRing : kMergeBytes) + kQBytes + (kMaxTopK + 1) * 4;
+  static int bytes(int table_cap) { return kFixed + table_cap * 4; }
+};
+
+// Byte offset of 16-byte chunk `c` of row `r` in a [rows][D] bf16 tile whose
+// chunks are XOR-swizzled by (r & 7) (conflict-free ldmatrix).
+template <int D>
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+  return static_cast<uint32_t>(r * (D * 2) + ((c ^ (r & 7)) << 4));
+}
+
+// grid (B * H_kv, n_split, T), block 128.
+template <int D, int G>
+__global__ void __launch_bounds__(128)
+attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__restrict__ ids,
+                  int k, const int64_t *__restrict__ doc_chunk_off, int n_docs,
+                  const int32_t *__restrict__ slots, int slot_chunks, int H_kv,
+                  const __nv_bfloat16 *__restrict__ Q, int T_tok,
+                  const __nv_bfloat16 *__restrict__ K_cache,
+                  const __nv_bfloat16 *__restrict__ V_cache, const int32_t *__restrict__ cache_len,
+                  int cap, int pos_offset, const float2 *__restrict__ rope, float scale_log2,
+                  int n_split, int table_cap, __nv_bfloat16 *__restrict__ O,
+                  float *__restrict__ part_o, float *__restrict__ part_ml) {
+  constexpr int CPR = D / 8;  // 16-byte chunks per row
+  using Sm = AttSmem<D>;
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint8_t *ring = sm;
+  uint8_t *qsm = sm + (Sm::kRing > Sm::kMergeBytes ? Sm::kRing : Sm::kMergeBytes);
+  int *pre = reinterpret_cast<int *>(qsm + Sm::kQBytes);
+  int *table = pre + (kMaxTopK + 1);
+
+  const int H_q = H_kv * G;
+  const int b = blockIdx.x / H_kv, g = blockIdx.x % H_kv;
+  const int split = blockIdx.y, i = blockIdx.z;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  const int n_mem = build_chunk_table(ids + static_cast<int64_t>(b) * k, k, doc_chunk_off, n_docs,
+                                      slots ? slots + static_cast<int64_t>(b) * k : nullptr,
+                                      slot_chunks, table, pre, table_cap);
+  const int j = cache_len[b] + i;
+  const bool overflow = j >= cap;
+  const int n_ctx = overflow ? 0 : n_mem + j + 1;
+  int per = (n_ctx + n_split - 1) / n_split;
+  per = (per + kAttRows - 1) / kAttRows * kAttRows;
+  const int x0 = split * per;
+  const int x1 = min(n_ctx, x0 + per);
+
+  // rotated query rows of the group -> qsm [16][D] (rows >= G are zero)
+  {
+    const int half = D / 2;
+    const __nv_bfloat16 *qb = Q + ((static_cast<int64_t>(b) * T_tok + i) * H_q + g * G) * D;
+    const float2 *cs = rope + static_cast<int64_t>(pos_offset + (overflow ? 0 : j)) * half;
+    for (int p = threadIdx.x; p < 16 * half; p += blockDim.x) {
+      const int r = p / half, e = p % half;
+      float lo = 0.0f, hi = 0.0f;
+      if (r < G) {
+        const float a = __bfloat162float(qb[r * D + e]);
+        const float c = __bfloat162float(qb[r * D + e + half]);
+        const float2 t = cs[e];
+        lo = a * t.x - c * t.y;
+        hi = c * t.x + a * t.y;
+      }
+      const __nv_bfloat16 blo = __float2bfloat16_rn(lo), bhi = __float2bfloat16_rn(hi);
+      *reinterpret_cast<__nv_bfloat16 *>(qsm + swz<D>(r, e / 8) + (e % 8) * 2) = blo;
+      *reinterpret_cast<__nv_bfloat16 *>(qsm + swz<D>(r, (e + half) / 8) + (e % 8) * 2) = bhi;
+    }
+  }
+  __syncthreads();
+
+  // A fragments of Q for every k-step
+  uint32_t qa[D / 16][4];
+  {
+    const uint32_t qbase = smem_u32(qsm);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int r = lane & 15, c = 2 * kk + (lane >> 4);
+      ldsm_x4(qbase + swz<D>(r, c), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+    }
+  }
+
+  const int64_t kv = static_cast<int64_t>(H_kv) * D;
+  uint8_t *wbuf = ring + warp * Sm::kWarpBytes;
+  // issue the loads of the block starting at context row x into stage s
+  auto issue = [&](int x, int s) {
+    uint8_t *kb = wbuf + s * 2 * Sm::kBlockBytes;
+    uint8_t *vb = kb + Sm::kBlockBytes;
+#pragma unroll
+    for (int u = 0; u < kAttRows * CPR / 32; ++u) {
+      const int idx = lane + 32 * u;
+      const int r = idx / CPR, c = idx % CPR;
+      const int xr = x + r;
+      const __nv_bfloat16 *ks = K_cache, *vs = V_cache;
+      bool ok = xr < x1;
+      if (ok) {
+        if (xr < n_mem) {
+          ks = content + static_cast<int64_t>(table[xr]) * 2 * kv + g * D;
+          vs = ks + kv;
+        } else {
+          const int64_t row = (static_cast<int64_t>(b) * cap + (xr - n_mem)) * kv + g * D;
+          ks = K_cache + row;
+          vs = V_cache + row;
+        }
+      }
+      cp_async_16(smem_u32(kb + swz<D>(r, c)), ks + c * 8, ok);
+      cp_async_16(smem_u32(vb + swz<D>(r, c)), vs + c * 8, ok);
+    }
+    cp_async_commit();
+  };
+
+  float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 domain) of rows g8 and g8+8
+  float l0 = 0.0f, l1 = 0.0f;
+  float acc[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[n][e] = 0.0f;
+
+  const int nblk = (x1 > x0) ? (x1 - x0 + kAttRows - 1) / kAttRows : 0;
+  int s = 0;
+  if (warp < nblk) issue(x0 + warp * kAttRows, 0);
+  for (int bi = warp; bi < nblk; bi += kAttWarps) {
+    const int x = x0 + bi * kAttRows;
+    if (bi + kAttWarps < nblk) {
+      issue(x + kAttWarps * kAttRows, s ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncwarp();
+    const uint32_t kb = smem_u32(wbuf + s * 2 * Sm::kBlockBytes);
+    const uint32_t vb = kb + Sm::kBlockBytes;
+
+    // S = Q K^T over 16 context rows (two n8 tiles)
+    float sc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[nt][e] = 0.0f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int r = (lane & 7) + ((lane >> 4) << 3), c = 2 * kk + ((lane >> 3) & 1);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(kb + swz<D>(r, c), b0, b1, b2, b3);
+      mma_bf16_16816(sc[0], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
+      mma_bf16_16816(sc[1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
+    }
+    // scale to log2 units, mask rows past the split end
+    float bm0 = -INFINITY, bm1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int col = x + nt * 8 + (lane & 3) * 2 + e;
+        const bool ok = col < x1;
+        sc[nt][e] = ok ? sc[nt][e] * scale_log2 : -INFINITY;
+        sc[nt][2 + e] = ok ? sc[nt][2 + e] * scale_log2 : -INFINITY;
+        bm0 = fmaxf(bm0, sc[nt][e]);
+        bm1 = fmaxf(bm1, sc[nt][2 + e]);
+      }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, o));
+      bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, o));
+    }
+    const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
+    const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
+    const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
+    const float al0 = exp2f(m0 - base0), al1 = exp2f(m1 - base1);
+    m0 = mn0;
+    m1 = mn1;
+    float ps0 = 0.0f, ps1 = 0.0f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        sc[nt][e] = exp2f(sc[nt][e] - base0);
+        sc[nt][2 + e] = exp2f(sc[nt][2 + e] - base1);
+        ps0 += sc[nt][e];
+        ps1 += sc[nt][2 + e];
+      }
+    l0 = l0 * al0 + ps0;
+    l1 = l1 * al1 + ps1;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      acc[n][0] *= al0;
+      acc[n][1] *= al0;
+      acc[n][2] *= al1;
+      acc[n][3] *= al1;
+    }
+    // O += P V
+    const uint32_t pa0 = pack_bf16x2(sc[0][0], sc[0][1]);
+    const uint32_t pa1 = pack_bf16x2(sc[0][2], sc[0][3]);
+    const uint32_t pa2 = pack_bf16x2(sc[1][0], sc[1][1]);
+    const uint32_t pa3 = pack_bf16x2(sc[1][2], sc[1][3]);
+#pragma unroll
+    for (int dp = 0; dp < D / 16; ++dp) {
+      const int r = (lane & 7) + (((lane >> 3) & 1) << 3), c = 2 * dp + (lane >> 4);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_trans(vb + swz<D>(r, c), b0, b1, b2, b3);
+      mma_bf16_16816(acc[2 * dp], pa0, pa1, pa2, pa3, b0, b1);
+      mma_bf16_16816(acc[2 * dp + 1], pa0, pa1, pa2, pa3, b2, b3);
+    }
+    __syncwarp();
+    s ^= 1;
+  }
+
+  // per-row totals across the 4 lanes of a row group
+#pragma unroll
+  for (int o = 1; o <= 2; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  __syncthreads();  // every warp is done with the ring: reuse it for the merge
+  float *mo = reinterpret_cast<float *>(ring);  // [warp][16][D + 2]: D outputs, m, l
+  {
+    const int r0 = lane >> 2;
+    float *row0 = mo + (warp * 16 + r0) * (D + 2);
+    float *row1 = mo + (warp * 16 + r0 + 8) * (D + 2);
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      const int col = n * 8 + (lane & 3) * 2;
+      row0[col] = acc[n][0];
+      row0[col + 1] = acc[n][1];
+      row1[col] = acc[n][2];
+      row1[col + 1] = acc[n][3];
+    }
+    if ((lane & 3) == 0) {
+      row0[D] = m0;
+      row0[D + 1] = l0;
+      row1[D] = m1;
+      row1[D + 1] = l1;
+    }
+  }
+  __syncthreads();
+  for (int p = threadIdx.x; p < G * D; p += blockDim.x) {
+    const int r = p / D, e = p % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kAttWarps; ++w) M = fmaxf(M, mo[(w * 16 + r) * (D + 2) + D]);
+    const float base = M == -INFINITY ? 0.0f : M;
+    float L = 0.0f, acc_o = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kAttWarps; ++w) {
+      const float *row = mo + (w * 16 + r) * (D + 2);
+      const float f = exp2f(row[D] - base);
+      L += row[D + 1] * f;
+      acc_o += row[e] * f;
+    }
+    const int h = g * G + r;
+    const int64_t orow = (static_cast<int64_t>(b) * T_tok + i) * H_q + h;
+    if (n_split == 1) {
+      O[orow * D + e] = __float2bfloat16_rn(L > 0.0f ? acc_o / L : 0.0f);
+    } else {
+      part_o[(orow * n_split + split) * D + e] = acc_o;
+      if (e == 0) {
+        part_ml[(orow * n_split + split) * 2] = M;
+        part_ml[(orow * n_split + split) * 2 + 1] = L;
+      }
+    }
+  }
+}
+
+// grid (B * T * H_q), block D: merge the context splits.  Partial maxima are
+// in log2 units.  Also advances cache_len[b] by T (one thread per query).
+__global__ void attend_combine_kernel(const float *__restrict__ part_o,
+                                      const float *__restrict__ part_ml, int n_split, int D,
+                                      __nv_bfloat16 *__restrict__ O) {
+  const int64_t orow = blockIdx.x;
+  const float *ml = part_ml + orow * n_split * 2;
+  float M = -INFINITY;
+  for (int s = 0; s < n_split; ++s) M = fmaxf(M, ml[2 * s]);
+  const float base = M == -INFINITY ? 0.0f : M;
+  for (int e = threadIdx.x; e < D; e += blockDim.x) {
+    float L = 0.0f, acc = 0.0f;
+    for (int s = 0; s < n_split; ++s) {
+      const float f = exp2f(ml[2 * s] - base);
+      L += ml[2 * s + 1] * f;
+      acc += part_o[(orow * n_split + s) * D + e] * f;
+    }
+    O[orow * D + e] = __float2bfloat16_rn(L > 0.0f ? acc / L : 0.0f);
+  }
+}
+
+__global__ void advance_kernel(int32_t *__restrict__ cache_len, int B, int T_tok, int cap) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) cache_len[b] = min(cache_len[b] + T_tok, cap);
+}
+
+}  // namespace msa

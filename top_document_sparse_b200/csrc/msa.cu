@@ -1,0 +1,654 @@
+// msa.cu -- the C ABI of libmsa.so (declared in include/msa.h): host-side
+// validation and orchestration of the MSA kernels.  Every kernel lives in the
+// headers included below; this file is the single translation unit.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+
+#include "attend.cuh"
+#include "common.cuh"
+#include "pool.cuh"
+#include "route.cuh"
+#include "topk.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+msa_status fail(msa_status s, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+msa_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(MSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define MSA_CUDA(call)                                 \
+  do {                                                 \
+    cudaError_t e_ = (call);                           \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+#define MSA_LAUNCHED(what)                              \
+  do {                                                  \
+    cudaError_t e_ = cudaGetLastError();                \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what);  \
+  } while (0)
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+int round32(int x) { return (x + 31) / 32 * 32; }
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+int max_dyn_smem() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (n <= 0) n = 232448;
+  }
+  return n;
+}
+
+// ---------------------------------------------------------------- TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [rows][cols] array, box {64 cols, box_rows},
+// 128-byte swizzle, out-of-range rows read as zero.
+msa_status make_map_bf16(CUtensorMap *map, const void *base, int64_t rows, int64_t cols,
+                         int box_rows) {
+  auto fn = encode_tiled();
+  if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MSA_OK;
+}
+
+// ---------------------------------------------------------------- helpers
+size_t elem_size(msa_dtype t) { return t == MSA_BF16 ? 2 : 4; }
+
+int topk_splits(int n_docs) { return (n_docs + msa::kTopkSlice - 1) / msa::kTopkSlice; }
+
+// context splits of one decode attention launch: enough CTAs to fill the GPU
+int attend_splits(int B, int T, int H_kv, int64_t max_ctx) {
+  const int64_t ctas = static_cast<int64_t>(B) * T * H_kv;
+  const int64_t want = 6LL * num_sms();
+  if (ctas >= want) return 1;
+  int64_t s = (want + ctas - 1) / ctas;
+  const int64_t by_len = std::max<int64_t>(1, (max_ctx + 63) / 64);
+  return static_cast<int>(std::min<int64_t>(std::min<int64_t>(s, by_len), 32));
+}
+
+struct AttendPlan {
+  int n_split = 1;
+  int table_cap = 0;
+  size_t part_o = 0, part_ml = 0;  // byte offsets in the workspace
+  size_t bytes = 0;
+};
+
+AttendPlan plan_attend(const msa_memory *mem, int B, int T, int k, int H_q, int cap) {
+  AttendPlan p;
+  const int64_t max_mem = static_cast<int64_t>(k) * mem->max_doc_chunks;
+  p.table_cap = static_cast<int>(std::min<int64_t>(max_mem, msa::kMaxMemRows));
+  if (mem->dtype == MSA_BF16) {
+    p.n_split = attend_splits(B, T, mem->H_kv, max_mem + cap);
+    if (p.n_split > 1) {
+      const size_t rows = static_cast<size_t>(B) * T * H_q * p.n_split;
+      p.part_o = 0;
+      p.part_ml = round256(rows * mem->D * 4);
+      p.bytes = p.part_ml + round256(rows * 2 * 4);
+    }
+  }
+  return p;
+}
+
+struct RoutePlan {
+  size_t qhat = 0, cand = 0, bytes = 0;
+  int n_split = 1;
+};
+
+RoutePlan plan_route(const msa_memory *mem, int B, int T, int k) {
+  RoutePlan p;
+  const size_t W = static_cast<size_t>(mem->H_r) * mem->d_r;
+  p.qhat = 0;
+  p.cand = round256(static_cast<size_t>(B) * T * W * elem_size(mem->dtype));
+  p.n_split = topk_splits(mem->n_docs);
+  p.bytes = p.cand + (p.n_split > 1 ? round256(static_cast<size_t>(B) * p.n_split * k * 8) : 0);
+  return p;
+}
+
+template <int NT>
+msa_status launch_route_mma(const msa_memory *mem, const void *keys, const void *qhat, int R,
+                            int T, float *state, cudaStream_t st) {
+  const int W = mem->H_r * mem->d_r;
+  CUtensorMap tmK, tmQ;
+  msa_status s = make_map_bf16(&tmK, keys, mem->n_chunks, W, msa::kRouteTileC);
+  if (s != MSA_OK) return s;
+  s = make_map_bf16(&tmQ, qhat, R, W, NT);
+  if (s != MSA_OK) return s;
+  const int maxs = max_dyn_smem();
+  int stages = 8;
+  while (stages > 2 && msa::RouteLayout<NT>::bytes(W, stages) > static_cast<size_t>(maxs)) --stages;
+  const size_t smem = msa::RouteLayout<NT>::bytes(W, stages);
+  if (smem > static_cast<size_t>(maxs))
+    return fail(MSA_ERR_UNSUPPORTED, "router width %d needs %zu B of shared memory", W, smem);
+  auto kern = msa::route_mma_kernel<NT>;
+  MSA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int n_ct = static_cast<int>((mem->n_chunks + msa::kRouteTileC - 1) / msa::kRouteTileC);
+  const int n_rt = (R + NT - 1) / NT;
+  const int64_t n_tiles = static_cast<int64_t>(n_ct) * n_rt;
+  if (n_tiles > INT32_MAX) return fail(MSA_ERR_UNSUPPORTED, "too many route tiles");
+  const int grid = static_cast<int>(std::min<int64_t>(n_tiles, num_sms()));
+  kern<<<grid, 160, smem, st>>>(tmK, tmQ, mem->n_chunks, R, W, T, 1.0f / mem->H_r,
+                                mem->d_chunk_doc, mem->n_docs, state, n_ct,
+                                static_cast<int>(n_tiles), stages);
+  MSA_LAUNCHED("route_mma_kernel");
+  return MSA_OK;
+}
+
+msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, int B, int T, int k,
+                      const uint8_t *exclude, float *state, int32_t *ids, float *scores,
+                      void *ws, size_t ws_bytes, cudaStream_t st) {
+  if (!mem) return fail(MSA_ERR_INVALID_ARG, "null memory");
+  if (B < 1 || T < 0) return fail(MSA_ERR_INVALID_ARG, "batch must be >= 1 and tokens >= 0");
+  if (k < 1 || k > mem->n_docs || k > msa::kMaxTopK)
+    return fail(MSA_ERR_INVALID_ARG, "k=%d must be in [1, min(n_docs=%d, %d)]", k, mem->n_docs,
+                msa::kMaxTopK);
+  if (!state || !ids || !scores) return fail(MSA_ERR_INVALID_ARG, "null state/ids/scores");
+  if (T > 0 && (!keys || !Qr)) return fail(MSA_ERR_INVALID_ARG, "null router keys or Qr");
+  if (!aligned16(keys) || !aligned16(Qr) || !aligned16(ws))
+    return fail(MSA_ERR_INVALID_ARG, "router keys, Qr and workspace must be 16-byte aligned");
+  const RoutePlan plan = plan_route(mem, B, T, k);
+  if (plan.n_split * k > msa::kTopkSlice)
+    return fail(MSA_ERR_UNSUPPORTED, "top-k merge of %d candidates is too large",
+                plan.n_split * k);
+  if (ws_bytes < plan.bytes || (plan.bytes > 0 && !ws))
+    return fail(MSA_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, plan.bytes);
+  const int64_t R64 = static_cast<int64_t>(B) * T;
+  if (R64 > INT32_MAX / 2) return fail(MSA_ERR_UNSUPPORTED, "too many query rows");
+  const int R = static_cast<int>(R64);
+  const int W = mem->H_r * mem->d_r;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  if (R > 0) {
+    const int thr = round32(W / 4);
+    if (mem->dtype == MSA_BF16) {
+      auto *qh = reinterpret_cast<__nv_bfloat16 *>(wsb + plan.qhat);
+      msa::qnorm_kernel<__nv_bfloat16><<<R, thr, 0, st>>>(
+          static_cast<const __nv_bfloat16 *>(Qr), W, mem->d_r, qh);
+      MSA_LAUNCHED("qnorm_kernel");
+      msa_status s;
+      if (R <= 16)
+        s = launch_route_mma<16>(mem, keys, qh, R, T, state, st);
+      else if (R <= 32)
+        s = launch_route_mma<32>(mem, keys, qh, R, T, state, st);
+      else
+        s = launch_route_mma<64>(mem, keys, qh, R, T, state, st);
+      if (s != MSA_OK) return s;
+    } else {
+      auto *qh = reinterpret_cast<float *>(wsb + plan.qhat);
+      msa::qnorm_kernel<float><<<R, thr, 0, st>>>(static_cast<const float *>(Qr), W, mem->d_r, qh);
+      MSA_LAUNCHED("qnorm_kernel");
+      dim3 grid(static_cast<unsigned>((mem->n_chunks + 31) / 32), static_cast<unsigned>((R + 31) / 32));
+      if (grid.y > 65535) return fail(MSA_ERR_UNSUPPORTED, "too many query rows for fp32 route");
+      msa::route_simt_kernel<float><<<grid, 256, 0, st>>>(
+          static_cast<const float *>(keys), qh, mem->n_chunks, R, W, T, 1.0f / mem->H_r,
+          mem->d_chunk_doc, mem->n_docs, state);
+      MSA_LAUNCHED("route_simt_kernel");
+    }
+  }
+  auto *cand = reinterpret_cast<unsigned long long *>(wsb + plan.cand);
+  if (B > 65535) return fail(MSA_ERR_UNSUPPORTED, "batch too large for top-k");
+  msa::topk_partial_kernel<<<dim3(plan.n_split, B), msa::kTopkThreads, 0, st>>>(
+      state, exclude, mem->n_docs, k, plan.n_split, cand, ids, scores);
+  MSA_LAUNCHED("topk_partial_kernel");
+  if (plan.n_split > 1) {
+    msa::topk_merge_kernel<<<B, msa::kTopkThreads, 0, st>>>(cand, plan.n_split * k, k, ids, scores);
+    MSA_LAUNCHED("topk_merge_kernel");
+  }
+  return MSA_OK;
+}
+
+template <int D, int G>
+msa_status launch_attend_mma(const msa_memory *mem, const void *content, const int32_t *ids,
+                             const int32_t *slots, int slot_chunks, int B, int k, int T,
+                             const void *Q, const void *Kc, const void *Vc,
+                             const int32_t *cache_len, int cap, int pos_offset,
+                             const AttendPlan &plan, void *O, void *ws, cudaStream_t st) {
+  using Sm = msa::AttSmem<D>;
+  const int smem = Sm::bytes(plan.table_cap);
+  auto kern = msa::attend_mma_kernel<D, G>;
+  MSA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  float *part_o = plan.n_split > 1 ? reinterpret_cast<float *>(wsb + plan.part_o) : nullptr;
+  float *part_ml = plan.n_split > 1 ? reinterpret_cast<float *>(wsb + plan.part_ml) : nullptr;
+  const float scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)) * 1.4426950408889634);
+  dim3 grid(static_cast<unsigned>(B * mem->H_kv), plan.n_split, T);
+  kern<<<grid, 128, smem, st>>>(
+      static_cast<const __nv_bfloat16 *>(content), ids, k, mem->d_doc_chunk_off, mem->n_docs, slots,
+      slot_chunks, mem->H_kv, static_cast<const __nv_bfloat16 *>(Q), T,
+      static_cast<const __nv_bfloat16 *>(Kc), static_cast<const __nv_bfloat16 *>(Vc), cache_len,
+      cap, pos_offset, mem->d_rope, scale_log2, plan.n_split, plan.table_cap,
+      static_cast<__nv_bfloat16 *>(O), part_o, part_ml);
+  MSA_LAUNCHED("attend_mma_kernel");
+  if (plan.n_split > 1) {
+    msa::attend_combine_kernel<<<static_cast<unsigned>(static_cast<int64_t>(B) * T * mem->H_kv * G),
+                                 D, 0, st>>>(part_o, part_ml, plan.n_split, D,
+                                             static_cast<__nv_bfloat16 *>(O));
+    MSA_LAUNCHED("attend_combine_kernel");
+  }
+  return MSA_OK;
+}
+
+template <int D>
+msa_status dispatch_group(int G, const msa_memory *mem, const void *content, const int32_t *ids,
+                          const int32_t *slots, int slot_chunks, int B, int k, int T,
+                          const void *Q, const void *Kc, const void *Vc, const int32_t *cache_len,
+                          int cap, int pos_offset, const AttendPlan &plan, void *O, void *ws,
+                          cudaStream_t st) {
+#define MSA_G(g)                                                                                  \
+  case g:                                                                                         \
+    return launch_attend_mma<D, g>(mem, content, ids, slots, slot_chunks, B, k, T, Q, Kc, Vc,     \
+                                   cache_len, cap, pos_offset, plan, O, ws, st);
+  switch (G) {
+    MSA_G(1) MSA_G(2) MSA_G(4) MSA_G(8) MSA_G(16)
+    default:
+      return fail(MSA_ERR_UNSUPPORTED, "GQA group %d (must be 1, 2, 4, 8 or 16)", G);
+  }
+#undef MSA_G
+}
+
+msa_status attend_impl(const msa_memory *mem, const void *content, const int32_t *ids,
+                       const int32_t *slots, int slot_chunks, int B, int k, int T, int H_q,
+                       const void *Q, const void *K_new, const void *V_new, void *K_cache,
+                       void *V_cache, int32_t *cache_len, int cap, int pos_offset, void *O,
+                       void *ws, size_t ws_bytes, cudaStream_t st) {
+  if (!mem) return fail(MSA_ERR_INVALID_ARG, "null memory");
+  if (B < 1 || T < 1) return fail(MSA_ERR_INVALID_ARG, "batch and tokens must be >= 1");
+  if (k < 0 || k > msa::kMaxTopK) return fail(MSA_ERR_INVALID_ARG, "k=%d out of range", k);
+  if (H_q < mem->H_kv || H_q % mem->H_kv != 0)
+    return fail(MSA_ERR_INVALID_ARG, "n_q_heads=%d must be a multiple of n_kv_heads=%d", H_q,
+                mem->H_kv);
+  if (H_q > 16 * 32) return fail(MSA_ERR_UNSUPPORTED, "too many query heads");
+  if (cap < 1 || pos_offset < 0 ||
+      static_cast<int64_t>(pos_offset) + cap > mem->max_local_position)
+    return fail(MSA_ERR_INVALID_ARG,
+                "pos_offset=%d + cache_capacity=%d must be <= max_local_position=%d", pos_offset,
+                cap, mem->max_local_position);
+  if (!content || (k > 0 && !ids) || !Q || !K_new || !V_new || !K_cache || !V_cache ||
+      !cache_len || !O)
+    return fail(MSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(content) || !aligned16(Q) || !aligned16(K_new) || !aligned16(V_new) ||
+      !aligned16(K_cache) || !aligned16(V_cache) || !aligned16(O) || !aligned16(ws))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (static_cast<int64_t>(k) * mem->max_doc_chunks > msa::kMaxMemRows)
+    return fail(MSA_ERR_UNSUPPORTED, "k * max_doc_chunks = %lld exceeds %d retrieved rows",
+                (long long)k * mem->max_doc_chunks, msa::kMaxMemRows);
+  if (static_cast<int64_t>(B) * T > 2147483647LL / 64)
+    return fail(MSA_ERR_UNSUPPORTED, "batch * tokens too large");
+  const AttendPlan plan = plan_attend(mem, B, T, k, H_q, cap);
+  if (ws_bytes < plan.bytes || (plan.bytes > 0 && !ws))
+    return fail(MSA_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, plan.bytes);
+  const int D = mem->D, H_kv = mem->H_kv;
+  // 1. append the new tokens (K rotated at pos_offset + j)
+  const int athr = round32(H_kv * D / 8);
+  if (athr > 1024) return fail(MSA_ERR_UNSUPPORTED, "n_kv_heads * head_dim too large");
+  if (mem->dtype == MSA_BF16) {
+    msa::append_kernel<__nv_bfloat16><<<B * T, athr, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(K_new), static_cast<const __nv_bfloat16 *>(V_new), T,
+        H_kv, D, static_cast<__nv_bfloat16 *>(K_cache), static_cast<__nv_bfloat16 *>(V_cache),
+        cache_len, cap, pos_offset, mem->d_rope);
+  } else {
+    msa::append_kernel<float><<<B * T, athr, 0, st>>>(
+        static_cast<const float *>(K_new), static_cast<const float *>(V_new), T, H_kv, D,
+        static_cast<float *>(K_cache), static_cast<float *>(V_cache), cache_len, cap, pos_offset,
+        mem->d_rope);
+  }
+  MSA_LAUNCHED("append_kernel");
+  // 2. attention over [memory rows | causal local rows]
+  const int G = H_q / H_kv;
+  msa_status s = MSA_OK;
+  if (mem->dtype == MSA_BF16) {
+    if (D == 128)
+      s = dispatch_group<128>(G, mem, content, ids, slots, slot_chunks, B, k, T, Q, K_cache,
+                              V_cache, cache_len, cap, pos_offset, plan, O, ws, st);
+    else
+      s = dispatch_group<64>(G, mem, content, ids, slots, slot_chunks, B, k, T, Q, K_cache,
+                             V_cache, cache_len, cap, pos_offset, plan, O, ws, st);
+  } else {
+    if (H_q > 16) return fail(MSA_ERR_UNSUPPORTED, "fp32 attention supports <= 16 query heads");
+    const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+    const int thr = H_q * 32;
+    if (D == 128)
+      msa::attend_simt_kernel<float, 128><<<B * T, thr, 0, st>>>(
+          static_cast<const float *>(content), ids, k, mem->d_doc_chunk_off, mem->n_docs, slots,
+          slot_chunks, H_kv, H_q, static_cast<const float *>(Q), T,
+          static_cast<const float *>(K_cache), static_cast<const float *>(V_cache), cache_len, cap,
+          pos_offset, mem->d_rope, scale, static_cast<float *>(O));
+    else
+      msa::attend_simt_kernel<float, 64><<<B * T, thr, 0, st>>>(
+          static_cast<const float *>(content), ids, k, mem->d_doc_chunk_off, mem->n_docs, slots,
+          slot_chunks, H_kv, H_q, static_cast<const float *>(Q), T,
+          static_cast<const float *>(K_cache), static_cast<const float *>(V_cache), cache_len, cap,
+          pos_offset, mem->d_rope, scale, static_cast<float *>(O));
+    MSA_LAUNCHED("attend_simt_kernel");
+  }
+  if (s != MSA_OK) return s;
+  // 3. the cache now holds T more rows
+  msa::advance_kernel<<<(B + 255) / 256, 256, 0, st>>>(cache_len, B, T, cap);
+  MSA_LAUNCHED("advance_kernel");
+  return MSA_OK;
+}
+
+}  // namespace
+
+// ===================================================================== C ABI
+extern "C" {
+
+int32_t msa_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+const char *msa_status_string(msa_status s) {
+  switch (s) {
+    case MSA_OK: return "ok";
+    case MSA_ERR_INVALID_ARG: return "invalid argument";
+    case MSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case MSA_ERR_CUDA: return "CUDA error";
+    case MSA_ERR_OUT_OF_MEMORY: return "out of memory";
+    case MSA_ERR_TIMEOUT: return "device wait timed out";
+    case MSA_ERR_STATE: return "device bounds check fired";
+  }
+  return "unknown status";
+}
+
+const char *msa_last_error(void) { return g_last_error.c_str(); }
+
+msa_status msa_memory_create(const msa_memory_config *cfg, msa_memory **out) {
+  if (!cfg || !out) return fail(MSA_ERR_INVALID_ARG, "null config or output");
+  *out = nullptr;
+  if (cfg->n_docs < 1 || !cfg->doc_token_offsets)
+    return fail(MSA_ERR_INVALID_ARG, "n_docs must be >= 1 with token offsets");
+  if (cfg->dtype != MSA_F32 && cfg->dtype != MSA_BF16)
+    return fail(MSA_ERR_INVALID_ARG, "dtype must be MSA_F32 or MSA_BF16");
+  if (cfg->chunk_len < 2 || cfg->chunk_len > msa::kMaxChunkLen)
+    return fail(MSA_ERR_UNSUPPORTED, "chunk_len=%d must be in [2, %d]", cfg->chunk_len,
+                msa::kMaxChunkLen);
+  if (cfg->head_dim != 64 && cfg->head_dim != 128)
+    return fail(MSA_ERR_UNSUPPORTED, "head_dim=%d must be 64 or 128", cfg->head_dim);
+  if (cfg->n_kv_heads < 1 || cfg->n_kv_heads * cfg->head_dim > 8192)
+    return fail(MSA_ERR_UNSUPPORTED, "n_kv_heads=%d out of range", cfg->n_kv_heads);
+  if (!pow2(cfg->router_dim) || cfg->router_dim < 16 || cfg->router_dim > 128)
+    return fail(MSA_ERR_UNSUPPORTED, "router_dim=%d must be a power of two in [16, 128]",
+                cfg->router_dim);
+  const int W = cfg->n_router_heads * cfg->router_dim;
+  if (cfg->n_router_heads < 1 || W % 64 != 0 || W > 4096)
+    return fail(MSA_ERR_UNSUPPORTED,
+                "n_router_heads * router_dim = %d must be a multiple of 64 and <= 4096", W);
+  if (!(cfg->rope_theta > 1.0)) return fail(MSA_ERR_INVALID_ARG, "rope_theta must be > 1");
+  if (cfg->max_local_position < 1)
+    return fail(MSA_ERR_INVALID_ARG, "max_local_position must be >= 1");
+  auto m = new msa_memory();
+  m->n_docs = cfg->n_docs;
+  m->chunk_len = cfg->chunk_len;
+  m->H_kv = cfg->n_kv_heads;
+  m->D = cfg->head_dim;
+  m->H_r = cfg->n_router_heads;
+  m->d_r = cfg->router_dim;
+  m->dtype = cfg->dtype;
+  m->theta = cfg->rope_theta;
+  m->max_local_position = cfg->max_local_position;
+  m->doc_tok_off.assign(cfg->doc_token_offsets, cfg->doc_token_offsets + cfg->n_docs + 1);
+  m->doc_chunk_off.resize(cfg->n_docs + 1);
+  if (m->doc_tok_off[0] != 0) {
+    delete m;
+    return fail(MSA_ERR_INVALID_ARG, "doc_token_offsets[0] must be 0");
+  }
+  m->doc_chunk_off[0] = 0;
+  for (int d = 0; d < cfg->n_docs; ++d) {
+    const int64_t len = m->doc_tok_off[d + 1] - m->doc_tok_off[d];
+    if (len <= 0) {
+      delete m;
+      return fail(MSA_ERR_INVALID_ARG, "document %d is empty (offsets must increase)", d);
+    }
+    const int64_t nc = (len + m->chunk_len - 1) / m->chunk_len;
+    m->doc_chunk_off[d + 1] = m->doc_chunk_off[d] + nc;
+    m->max_doc_chunks = static_cast<int32_t>(std::max<int64_t>(m->max_doc_chunks, nc));
+    m->max_doc_tokens = std::max<int64_t>(m->max_doc_tokens, len);
+  }
+  m->n_tokens = m->doc_tok_off[cfg->n_docs];
+  m->n_chunks = m->doc_chunk_off[cfg->n_docs];
+  if (m->n_chunks >= INT32_MAX) {
+    delete m;
+    return fail(MSA_ERR_UNSUPPORTED, "too many chunks");
+  }
+  m->rope_len = static_cast<int32_t>(
+      std::max<int64_t>(m->max_doc_tokens, static_cast<int64_t>(m->max_local_position)));
+  cudaGetDevice(&m->device);
+
+  // host tables
+  std::vector<int32_t> chunk_doc(m->n_chunks);
+  for (int d = 0; d < cfg->n_docs; ++d)
+    for (int64_t c = m->doc_chunk_off[d]; c < m->doc_chunk_off[d + 1]; ++c) chunk_doc[c] = d;
+  const int half = m->D / 2;
+  std::vector<float2> rope(static_cast<size_t>(m->rope_len) * half);
+  for (int64_t p = 0; p < m->rope_len; ++p)
+    for (int i = 0; i < half; ++i) {
+      const double ang =
+          static_cast<double>(p) * std::pow(m->theta, -2.0 * static_cast<double>(i) / m->D);
+      rope[p * half + i] = make_float2(static_cast<float>(std::cos(ang)),
+                                       static_cast<float>(std::sin(ang)));
+    }
+  auto alloc = [&](void **p, size_t n) { return cudaMalloc(p, std::max<size_t>(n, 16)); };
+  if (alloc(reinterpret_cast<void **>(&m->d_chunk_doc), chunk_doc.size() * 4) != cudaSuccess ||
+      alloc(reinterpret_cast<void **>(&m->d_doc_tok_off), m->doc_tok_off.size() * 8) != cudaSuccess ||
+      alloc(reinterpret_cast<void **>(&m->d_doc_chunk_off), m->doc_chunk_off.size() * 8) != cudaSuccess ||
+      alloc(reinterpret_cast<void **>(&m->d_rope), rope.size() * sizeof(float2)) != cudaSuccess) {
+    cudaGetLastError();
+    msa_memory_destroy(m);
+    return fail(MSA_ERR_OUT_OF_MEMORY, "could not allocate the memory tables");
+  }
+  if (cudaMemcpy(m->d_chunk_doc, chunk_doc.data(), chunk_doc.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(m->d_doc_tok_off, m->doc_tok_off.data(), m->doc_tok_off.size() * 8, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(m->d_doc_chunk_off, m->doc_chunk_off.data(), m->doc_chunk_off.size() * 8, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(m->d_rope, rope.data(), rope.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaError_t e = cudaGetLastError();
+    msa_memory_destroy(m);
+    return cuda_fail(e, "uploading memory tables");
+  }
+  *out = m;
+  return MSA_OK;
+}
+
+msa_status msa_memory_destroy(msa_memory *mem) {
+  if (!mem) return fail(MSA_ERR_INVALID_ARG, "null memory");
+  cudaFree(mem->d_chunk_doc);
+  cudaFree(mem->d_doc_tok_off);
+  cudaFree(mem->d_doc_chunk_off);
+  cudaFree(mem->d_rope);
+  delete mem;
+  return MSA_OK;
+}
+
+msa_status msa_memory_get_info(const msa_memory *mem, msa_memory_info *out) {
+  if (!mem || !out) return fail(MSA_ERR_INVALID_ARG, "null argument");
+  const size_t es = elem_size(mem->dtype);
+  out->n_tokens = mem->n_tokens;
+  out->n_chunks = mem->n_chunks;
+  out->max_doc_chunks = mem->max_doc_chunks;
+  out->max_doc_tokens = mem->max_doc_tokens;
+  out->elem_bytes = es;
+  out->router_key_bytes = static_cast<size_t>(mem->n_chunks) * mem->H_r * mem->d_r * es;
+  out->content_bytes = static_cast<size_t>(mem->n_chunks) * 2 * mem->H_kv * mem->D * es;
+  out->doc_content_stride = static_cast<size_t>(mem->max_doc_chunks) * 2 * mem->H_kv * mem->D * es;
+  return MSA_OK;
+}
+
+msa_status msa_memory_doc_chunk_offsets(const msa_memory *mem, int64_t *out) {
+  if (!mem || !out) return fail(MSA_ERR_INVALID_ARG, "null argument");
+  std::copy(mem->doc_chunk_off.begin(), mem->doc_chunk_off.end(), out);
+  return MSA_OK;
+}
+
+msa_status msa_encode_memory(const msa_memory *mem, int32_t doc_begin, int32_t doc_count,
+                             const void *K, const void *V, const void *Kr, void *router_keys,
+                             void *content, void *router_mean, msa_stream stream) {
+  if (!mem) return fail(MSA_ERR_INVALID_ARG, "null memory");
+  if (doc_begin < 0 || doc_count < 1 || doc_count > mem->n_docs - doc_begin)
+    return fail(MSA_ERR_INVALID_ARG, "document range [%d, %d+%d) outside [0, %d)", doc_begin,
+                doc_begin, doc_count, mem->n_docs);
+  if (!K || !V || !Kr || !router_keys || !content)
+    return fail(MSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(K) || !aligned16(V) || !aligned16(Kr) || !aligned16(router_keys) ||
+      !aligned16(content) || !aligned16(router_mean))
+    return fail(MSA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t c0 = mem->doc_chunk_off[doc_begin];
+  const int64_t nc = mem->doc_chunk_off[doc_begin + doc_count] - c0;
+  const int64_t tok_base = mem->doc_tok_off[doc_begin];
+  if (nc > INT32_MAX) return fail(MSA_ERR_UNSUPPORTED, "too many chunks in one call");
+  const int WK = mem->H_kv * mem->D, WR = mem->H_r * mem->d_r;
+  const int thr_k = round32(WK / 8), thr_v = round32(WK / 4), thr_r = round32(WR / 4);
+  if (thr_v > 1024 || thr_r > 1024) return fail(MSA_ERR_UNSUPPORTED, "rows too wide");
+  const unsigned grid = static_cast<unsigned>(nc);
+#define MSA_ENCODE(T)                                                                             \
+  msa::pool_rope_kernel<T><<<grid, thr_k, 0, st>>>(                                               \
+      static_cast<const T *>(K), tok_base, mem->H_kv, mem->D, c0, mem->d_chunk_doc,               \
+      mem->d_doc_tok_off, mem->d_doc_chunk_off, mem->chunk_len, mem->d_rope,                      \
+      static_cast<T *>(content), 2LL * WK);                                                       \
+  MSA_LAUNCHED("pool_rope_kernel");                                                               \
+  msa::pool_plain_kernel<T, false><<<grid, thr_v, 0, st>>>(                                       \
+      static_cast<const T *>(V), tok_base, WK, c0, mem->d_chunk_doc, mem->d_doc_tok_off,          \
+      mem->d_doc_chunk_off, mem->chunk_len, static_cast<T *>(content), 2LL * WK, WK, mem->D,      \
+      nullptr);                                                                                   \
+  MSA_LAUNCHED("pool_plain_kernel(V)");                                                           \
+  msa::pool_plain_kernel<T, true><<<grid, thr_r, 0, st>>>(                                        \
+      static_cast<const T *>(Kr), tok_base, WR, c0, mem->d_chunk_doc, mem->d_doc_tok_off,         \
+      mem->d_doc_chunk_off, mem->chunk_len, static_cast<T *>(router_keys), WR, 0, mem->d_r,       \
+      static_cast<T *>(router_mean));                                                             \
+  MSA_LAUNCHED("pool_plain_kernel(Kr)");
+  if (mem->dtype == MSA_BF16) {
+    MSA_ENCODE(__nv_bfloat16)
+  } else {
+    MSA_ENCODE(float)
+  }
+#undef MSA_ENCODE
+  return MSA_OK;
+}
+
+msa_status msa_route_reset(float *state, int64_t count, msa_stream stream) {
+  if (!state || count < 1) return fail(MSA_ERR_INVALID_ARG, "null state or empty count");
+  const int64_t blocks = std::min<int64_t>((count + 255) / 256, 4096);
+  msa::fill_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                     reinterpret_cast<cudaStream_t>(stream)>>>(state, count, -INFINITY);
+  MSA_LAUNCHED("fill_kernel");
+  return MSA_OK;
+}
+
+size_t msa_route_workspace_size(const msa_memory *mem, int32_t batch, int32_t tokens, int32_t k) {
+  if (!mem || batch < 1 || tokens < 0 || k < 1) return 0;
+  return plan_route(mem, batch, tokens, k).bytes;
+}
+
+msa_status msa_route(const msa_memory *mem, const void *router_keys, const void *Qr, int32_t batch,
+                     int32_t tokens, int32_t k, const uint8_t *exclude, float *state, int32_t *ids,
+                     float *scores, void *workspace, size_t workspace_bytes, msa_stream stream) {
+  return route_impl(mem, router_keys, Qr, batch, tokens, k, exclude, state, ids, scores, workspace,
+                    workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t msa_attend_workspace_size(const msa_memory *mem, int32_t batch, int32_t tokens, int32_t k,
+                                 int32_t n_q_heads) {
+  if (!mem || batch < 1 || tokens < 1 || k < 0 || n_q_heads < 1) return 0;
+  return plan_attend(mem, batch, tokens, k, n_q_heads, mem->max_local_position).bytes;
+}
+
+msa_status msa_sparse_attend(const msa_memory *mem, const void *content, const int32_t *ids,
+                             int32_t batch, int32_t k, int32_t tokens, int32_t n_q_heads,
+                             const void *Q, const void *K_new, const void *V_new, void *K_cache,
+                             void *V_cache, int32_t *cache_len, int32_t cache_capacity,
+                             int32_t pos_offset, void *O, void *workspace, size_t workspace_bytes,
+                             msa_stream stream) {
+  return attend_impl(mem, content, ids, nullptr, 0, batch, k, tokens, n_q_heads, Q, K_new, V_new,
+                     K_cache, V_cache, cache_len, cache_capacity, pos_offset, O, workspace,
+                     workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t msa_step_workspace_size(const msa_memory *mem, int32_t batch, int32_t k, int32_t n_q_heads) {
+  if (!mem || batch < 1 || k < 1 || n_q_heads < 1) return 0;
+  return round256(plan_route(mem, batch, 1, k).bytes) +
+         plan_attend(mem, batch, 1, k, n_q_heads, mem->max_local_position).bytes;
+}
+
+msa_status msa_step(const msa_memory *mem, const void *router_keys, const void *content,
+                    const msa_decode_state *s, const void *Qr_tok, const void *Q_tok,
+                    const void *K_tok, const void *V_tok, void *O_tok, msa_stream stream) {
+  if (!mem || !s) return fail(MSA_ERR_INVALID_ARG, "null memory or decode state");
+  const size_t need = msa_step_workspace_size(mem, s->batch, s->top_k, s->n_q_heads);
+  if (s->workspace_bytes < need || !s->workspace)
+    return fail(MSA_ERR_INVALID_ARG, "decode workspace too small: %zu < %zu", s->workspace_bytes,
+                need);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t route_bytes = round256(plan_route(mem, s->batch, 1, s->top_k).bytes);
+  uint8_t *ws = static_cast<uint8_t *>(s->workspace);
+  msa_status r = route_impl(mem, router_keys, Qr_tok, s->batch, 1, s->top_k, nullptr, s->state,
+                            s->ids, s->scores, ws, route_bytes, st);
+  if (r != MSA_OK) return r;
+  return attend_impl(mem, content, s->ids, nullptr, 0, s->batch, s->top_k, 1, s->n_q_heads, Q_tok,
+                     K_tok, V_tok, s->k_cache, s->v_cache, s->cache_len, s->cache_capacity,
+                     s->pos_offset, O_tok, ws + route_bytes, s->workspace_bytes - route_bytes, st);
+}
+
+msa_status msa_device_error(uint32_t *bits, msa_stream stream) {
+  if (!bits) return fail(MSA_ERR_INVALID_ARG, "null output");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int v = 0, zero = 0;
+  MSA_CUDA(cudaMemcpyFromSymbolAsync(&v, msa::g_device_error, sizeof(v), 0,
+                                     cudaMemcpyDeviceToHost, st));
+  MSA_CUDA(cudaMemcpyToSymbolAsync(msa::g_device_error, &zero, sizeof(zero), 0,
+                                   cudaMemcpyHostToDevice, st));
+  MSA_CUDA(cudaStreamSynchronize(st));
+  *bits = v;
+  if (v & MSA_DEVERR_WAIT_TIMEOUT) return fail(MSA_ERR_TIMEOUT, "a device wait timed out");
+  if (v) return fail(MSA_ERR_STATE, "device bounds check fired (bits 0x%x)", v);
+  return MSA_OK;
+}
+
+}  // extern "C"
