@@ -1,0 +1,551 @@
+"""Benchmark: routed decode steps/s of the MSA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl msa|reference]
+                    [--workload mem1m_bf16] [--layers L]
+
+One step = one routed decode token for every query of the batch through every routed layer:
+route (cosine score of the new token against every pooled router key, running max, top-k) then
+sparse GQA attention over the retrieved documents' pooled K/V and the local cache, via msa_step.
+Inputs are synthetic (seeded Gaussians with planted relevant documents; see
+top_document_sparse_b200/inputs.py), resident in HBM before the timed region.  Each step reads
+every layer's router keys and attention context (~2.4 GB at the 1M-token workload), more than
+the 126 MB L2, so no L2 flush is needed between steps.  Multi-GPU runs are replicas (the memory
+and the batch are per GPU; weak scaling, no collective on the data path).
+
+Rank 0 prints one JSON line.  --impl reference times the fp64 CPU oracle on a bounded sample of
+the same workload instead (the reference arm: it is a deliberately slow program).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from top_document_sparse_b200 import inputs  # noqa: E402
+from top_document_sparse_b200.workloads import WORKLOADS  # noqa: E402
+
+METRIC = "routed decode steps/s at 1M & 100M-token memory; route_score HBM GB/s vs peak"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1024)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
+    ap.add_argument("--workload", default="mem1m_bf16")
+    ap.add_argument("--layers", type=int, default=0, help="routed layers (default: workload's)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        try:
+            self.dev = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            self.dev = str(device_index)
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.dev, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- GPU arm
+class LayerState:
+    pass
+
+
+def build_layers(w, n_layers, seed, msa, t_enc):
+    """Encode every routed layer's memory from seeded raw tokens (generated on the device in
+    document blocks), then prefill: route the query block and attend it."""
+    dev = "cuda"
+    off = inputs.doc_offsets(w, seed)
+    dt = inputs.torch_dtype(w.dtype)
+    B, T, k, H_q = w.batch, w.query_tokens, w.top_k, w.n_q_heads
+    cap = T + w.decode_steps
+    mem = msa.Memory(off, w.chunk_len, w.n_kv_heads, w.head_dim, w.n_router_heads, w.router_dim,
+                     dt, w.rope_theta, k + cap)
+    layers = []
+    block_docs = max(1, (1 << 18) // max(1, int(off[1] - off[0])))  # ~256K tokens per block
+    enc_bytes = 0
+    for l in range(n_layers):
+        L = LayerState()
+        L.rk = mem.new_router_keys()
+        L.ct = mem.new_content()
+        Qr, Q, Kn, Vn = inputs.queries(w, B, T, seed=seed * 1000 + 7 * l + 1, device=dev)
+        plants = inputs.choose_plants(w, off, B, T, w.planted_per_query, seed=seed * 1000 + l)
+        pb, pd, pc, pt = plants
+        for d0 in range(0, mem.n_docs, block_docs):
+            d1 = min(mem.n_docs, d0 + block_docs)
+            t0, t1 = int(off[d0]), int(off[d1])
+            K, V, Kr = inputs.raw_memory(w, t1 - t0, seed=(seed * 1000 + l) * 100003 + d0,
+                                         device=dev)
+            sel = (pd >= d0) & (pd < d1)
+            if sel.any():
+                inputs.plant(w, Kr, Qr, off, (pb[sel], pd[sel], pc[sel], pt[sel]),
+                             w.planted_cos, seed=seed * 1000 + l, tok_base=t0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            mem.encode(d0, d1 - d0, K, V, Kr, L.rk, L.ct)
+            e1.record()
+            t_enc.append((e0, e1))
+            enc_bytes += (K.numel() + V.numel() + Kr.numel()) * K.element_size()
+            del K, V, Kr
+        L.dec = msa.LayerDecode(mem, B, k, H_q, cap)
+        L.Qr_pre = Qr
+        L.prefill = (Q, Kn, Vn)
+        L.plants = plants
+        layers.append(L)
+    return mem, off, layers, enc_bytes
+
+
+def prefill(mem, w, layers, msa):
+    B, T, k, H_q = w.batch, w.query_tokens, w.top_k, w.n_q_heads
+    ws_r = msa.workspace(mem.route_workspace_size(B, T, k))
+    ws_a = msa.workspace(mem.attend_workspace_size(B, T, k, H_q))
+    O = torch.empty(B, T, H_q, w.head_dim, dtype=mem.dtype, device="cuda")
+    ev = []
+    for L in layers:
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        mem.route(L.rk, L.Qr_pre, k, L.dec.state, L.dec.ids, L.dec.scores, ws_r)
+        e1.record()
+        Q, Kn, Vn = L.prefill
+        mem.sparse_attend(L.ct, L.dec.ids, Q, Kn, Vn, L.dec.k_cache, L.dec.v_cache,
+                          L.dec.cache_len, L.dec.pos_offset, O, ws_a)
+        e2.record()
+        ev.append((e0, e1, e2))
+    torch.cuda.synchronize()
+    for L in layers:
+        L.state0 = L.dec.state.clone()
+        L.len0 = L.dec.cache_len.clone()
+        del L.prefill, L.Qr_pre
+    return ev
+
+
+def run_gpu(args, w, world, rank, local):
+    from top_document_sparse_b200 import msa
+    n_layers = args.layers or w.n_layers
+    B, k, H_q, D, H_kv = w.batch, w.top_k, w.n_q_heads, w.head_dim, w.n_kv_heads
+    W_r = w.n_router_heads * w.router_dim
+    S = w.decode_steps
+    es = 2 if w.dtype == "bf16" else 4
+    seed = 1234 + rank
+    t_enc = []
+    mem, off, layers, enc_bytes = build_layers(w, n_layers, seed, msa, t_enc)
+    pre_ev = prefill(mem, w, layers, msa)
+    enc_ms = sum(a.elapsed_time(b) for a, b in t_enc)
+    pre_route_ms = sum(a.elapsed_time(b) for a, b, _ in pre_ev)
+    pre_attn_ms = sum(b.elapsed_time(c) for _, b, c in pre_ev)
+    planted_ok = all(set(L.plants[1][L.plants[0] == b].tolist()) <=
+                     set(L.dec.ids[b].cpu().tolist()) for L in layers for b in range(B))
+
+    # decode inputs: [layer][position][batch][...] per field, so every (layer, position) view is
+    # a dense tensor msa_step can take directly
+    g = inputs.generator(seed + 99, "cuda")
+    dt = mem.dtype
+    Qr_all = inputs.gaussian((n_layers, S, B, w.n_router_heads, w.router_dim), g, "cuda", dt)
+    Q_all = inputs.gaussian((n_layers, S, B, H_q, D), g, "cuda", dt)
+    K_all = inputs.gaussian((n_layers, S, B, H_kv, D), g, "cuda", dt)
+    V_all = inputs.gaussian((n_layers, S, B, H_kv, D), g, "cuda", dt)
+    fields = [[(Qr_all[l, s], Q_all[l, s], K_all[l, s], V_all[l, s]) for s in range(S)]
+              for l in range(n_layers)]
+    out = torch.empty(n_layers, B, H_q * D, dtype=dt, device="cuda")
+
+    def reset():
+        for L in layers:
+            L.dec.state.copy_(L.state0)
+            L.dec.cache_len.copy_(L.len0)
+
+    def step(s, flds, o):
+        if s == 0:
+            reset()
+        for l, L in enumerate(layers):
+            Qr, Q, Kt, Vt = flds[l][s] if flds is not None else flds_static[l]
+            mem.step(L.rk, L.ct, L.dec, Qr, Q, Kt, Vt, o[l])
+
+    # CUDA graphs: one per decode position (inputs differ per position)
+    stream = torch.cuda.Stream()
+    graphs = []
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for s in range(S):  # eager warm pass through every position (also checks the calls)
+            step(s, fields, out)
+    torch.cuda.synchronize()
+    assert msa.device_error() == 0
+    for s in range(S):
+        gph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gph, stream=stream):
+            step(s, fields, out)
+        graphs.append(gph)
+    torch.cuda.synchronize()
+
+    K, Wm = args.steps, args.warmup
+    for i in range(Wm):
+        graphs[i % S].replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        cur = torch.cuda.current_stream()
+        e0.record(cur)
+        for i in range(Wm, Wm + K):
+            graphs[i % S].replay()
+        e1.record(cur)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_per_step = ms / K
+    assert msa.device_error() == 0
+
+    # ---------------------------------------------------------------- e2e through host buffers
+    e2e = None
+    if not args.no_e2e:
+        flds_static = [tuple(torch.empty_like(v) for v in fields[l][0]) for l in range(n_layers)]
+        hosts = [x.cpu().pin_memory() for x in (Qr_all, Q_all, K_all, V_all)]
+        host_fields = [[tuple(h[l, s] for h in hosts) for s in range(S)]
+                       for l in range(n_layers)]
+        out_host = torch.empty(out.shape, dtype=dt, pin_memory=True)
+        ids_host = torch.empty(n_layers, B, k, dtype=torch.int32, pin_memory=True)
+        g_e2e = []
+        for s0 in (0, 1):
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph, stream=stream):
+                step(s0, None, out)
+            g_e2e.append(gph)
+        torch.cuda.synchronize()
+        h2d = sum(v.numel() * v.element_size() for l in range(n_layers) for v in fields[l][0])
+        d2h = out.numel() * out.element_size() + ids_host.numel() * 4
+        K2 = min(K, 4 * S)
+        cur = torch.cuda.current_stream()
+
+        def e2e_step(i):
+            s = i % S
+            for l in range(n_layers):
+                for dst, src in zip(flds_static[l], host_fields[l][s]):
+                    dst.copy_(src, non_blocking=True)
+            g_e2e[0 if s == 0 else 1].replay()
+            out_host.copy_(out, non_blocking=True)
+            for l, L in enumerate(layers):
+                ids_host[l].copy_(L.dec.ids, non_blocking=True)
+
+        # position must restart at 0 with a reset: run a whole number of episodes
+        for i in range(min(Wm, S)):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(cur)
+        for i in range(K2):
+            e2e_step(i)
+        a1.record(cur)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms2 = max_over_ranks(a0.elapsed_time(a1), world)
+        e2e = {"value": round(world * K2 / (ms2 / 1e3), 2), "unit": "steps/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "tokens_per_s": round(world * K2 * B / (ms2 / 1e3), 1)}
+        del host_fields, hosts
+
+    # ---------------------------------------------------------------- per-kernel timing
+    # Route and attention called separately (what msa_step does inside), captured in graphs
+    # with external event-record nodes between them; one decode position per replay.
+    ws_r = msa.workspace(mem.route_workspace_size(B, 1, k))
+    ws_a = msa.workspace(mem.attend_workspace_size(B, 1, k, H_q))
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+           for _ in range(n_layers)]
+    prof_steps = list(range(0, S, max(1, S // 16)))
+    route_ms, attn_ms, attn_ctx = [], [], []
+    reset()
+    torch.cuda.synchronize()
+    for s in range(S):
+        gph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gph, stream=stream):
+            for l, L in enumerate(layers):
+                Qr, Q, Kt, Vt = fields[l][s]
+                evs[l][0].record()
+                mem.route(L.rk, Qr[:, None], k, L.dec.state, L.dec.ids, L.dec.scores, ws_r)
+                evs[l][1].record()
+                mem.sparse_attend(L.ct, L.dec.ids, Q[:, None], Kt[:, None], Vt[:, None],
+                                  L.dec.k_cache, L.dec.v_cache, L.dec.cache_len,
+                                  L.dec.pos_offset, out[l].view(B, 1, H_q, D), ws_a)
+                evs[l][2].record()
+        gph.replay()
+        torch.cuda.synchronize()
+        if s in prof_steps:
+            for l in range(n_layers):
+                route_ms.append(evs[l][0].elapsed_time(evs[l][1]))
+                attn_ms.append(evs[l][1].elapsed_time(evs[l][2]))
+                attn_ctx.append(w.query_tokens + s + 1)
+        del gph
+    assert msa.device_error() == 0
+
+    hbm, peak_kind = peaks()
+    n_mem_rows = k * w.chunks_per_doc
+    route_bytes = mem.n_chunks * W_r * es + 2 * B * mem.n_docs * 4 + B * W_r * es
+    route_gbs = route_bytes / (statistics.mean(route_ms) * 1e-3) / 1e9
+    attn_bytes = [B * H_kv * (n_mem_rows + c) * 2 * D * es + 2 * B * H_q * D * es for c in attn_ctx]
+    attn_gbs = statistics.mean(b / (t * 1e-3) / 1e9 for b, t in zip(attn_bytes, attn_ms))
+    step_bytes = n_layers * (route_bytes + statistics.mean(attn_bytes))
+    kernels = {
+        "route": {"ms_per_call": round(statistics.mean(route_ms), 5),
+                  "bytes_per_call": int(route_bytes), "achieved_gbs": round(route_gbs, 1),
+                  "frac": round(route_gbs / hbm, 4)},
+        "attend": {"ms_per_call": round(statistics.mean(attn_ms), 5),
+                   "bytes_per_call": int(statistics.mean(attn_bytes)),
+                   "achieved_gbs": round(attn_gbs, 1), "frac": round(attn_gbs / hbm, 4)},
+    }
+    dom = max(kernels, key=lambda n: kernels[n]["ms_per_call"])
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tr_path):
+        with open(tr_path) as f:
+            traffic = json.load(f).get(w.name, {}).get(dom)
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["achieved_gbs"],
+                "peak": hbm, "unit": "GB/s", "frac": kernels[dom]["frac"], "traffic": traffic,
+                "peak_source": peak_kind}
+    ceiling_ms = step_bytes / (hbm * 1e9) * 1e3
+    res = {
+        "metric": METRIC,
+        "value": round(world * K / (ms / 1e3), 2),
+        "unit": "steps/s",
+        "n_gpus": world, "steps": K, "warmup": Wm,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded N(0,1) K/V/K_r/Q with planted relevant documents)",
+        "config": {"workload": w.name, "n_docs": mem.n_docs, "memory_tokens": int(off[-1]),
+                   "chunks": int(mem.n_chunks), "layers": n_layers, "batch": B, "top_k": k,
+                   "query_tokens": w.query_tokens, "decode_positions": S,
+                   "heads": f"{H_q}q/{H_kv}kv x {D}, router {w.n_router_heads}x{w.router_dim}",
+                   "parallelism": f"replicas x{world}",
+                   "l2": "no flush: every step streams ~%.1f GB > 126 MB L2" % (step_bytes / 1e9),
+                   "cuda_graphs": True},
+        "tokens_per_s": round(world * K * B / (ms / 1e3), 1),
+        "roofline": roofline,
+        "kernels": kernels,
+        "step_roofline": {"bytes_per_step": int(step_bytes), "ceiling_ms": round(ceiling_ms, 5),
+                          "frac": round(ceiling_ms / ms_per_step, 4)},
+        "encode": {"gbs": round(enc_bytes / (enc_ms * 1e-3) / 1e9, 1), "ms": round(enc_ms, 2)},
+        "prefill": {"route_ms": round(pre_route_ms, 3), "attend_ms": round(pre_attn_ms, 3),
+                    "route_tflops": round(n_layers * 2 * B * w.query_tokens * mem.n_chunks * W_r
+                                          / (pre_route_ms * 1e-3) / 1e12, 1)},
+        "planted_retrieved": planted_ok,
+        "gpu_launches": None,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    # library kernels per layer and step: qnorm, route, top-k (+ merge over 4096-document
+    # slices), append, attention (+ split combine), advance
+    split = mem.attend_workspace_size(B, 1, k, H_q) > 0
+    per_layer = 3 + (1 if mem.n_docs > 4096 else 0) + 3 + (1 if split else 0)
+    res["gpu_launches"] = K * n_layers * per_layer
+    return res
+
+
+# ---------------------------------------------------------------------------- CPU baseline
+class OracleSample:
+    """The fp64 oracle on a bounded sample of the workload's decode step: one decode token for a
+    few queries of one layer, routed against a slice of the documents, top-k over all documents,
+    attention over k retrieved documents plus the local rows.  ``step()`` times one sampled step
+    and extrapolates it linearly to the whole step (every query, layer and document)."""
+
+    def __init__(self, w, seed, n_docs_sample, queries):
+        import oracle
+        self.oracle, self.w = oracle, w
+        off_full = inputs.doc_offsets(w, seed)
+        self.n_docs = off_full.size - 1
+        self.nd = nd = min(n_docs_sample, self.n_docs)
+        off = off_full[:nd + 1]
+        self.B, T = queries, w.query_tokens
+        K, V, Kr = inputs.raw_memory(w, int(off[-1]), seed, "cpu")
+        self.Qr, self.Q, self.Kn, self.Vn = inputs.queries(w, self.B, T + 1, seed + 1, "cpu")
+        self.cho = oracle.doc_chunks(off, w.chunk_len)
+        self.Kb, self.Vb, self.Krb = oracle.encode(K, V, Kr, off, w.chunk_len, w.rope_theta)
+        self.state = oracle.route(self.Qr[:, :T], self.Krb, self.cho)
+        rng = np.random.default_rng(0)
+        self.full_state = np.concatenate(
+            [self.state, rng.uniform(-0.2, 0.2, size=(self.B, self.n_docs - nd))], axis=1)
+        kk = min(w.top_k, nd)
+        self.ids = np.stack([rng.choice(nd, size=kk, replace=False)
+                             for _ in range(self.B)]).astype(np.int32)
+        self.cores = len(os.sched_getaffinity(0))
+
+    def step(self):
+        o, w, T = self.oracle, self.w, self.w.query_tokens
+        t0 = time.perf_counter()
+        o.route(self.Qr[:, T], self.Krb, self.cho, self.state)
+        t1 = time.perf_counter()
+        o.topk(self.full_state, w.top_k)
+        t2 = time.perf_counter()
+        o.attend(self.Q[:, T:T + 1], self.Kn, self.Vn, T, self.Kb, self.Vb, self.cho, self.ids,
+                 w.top_k, w.rope_theta)
+        t3 = time.perf_counter()
+        per_q = ((t1 - t0) * (self.n_docs / self.nd) + (t2 - t1) + (t3 - t2)) / self.B
+        return per_q * w.batch * w.n_layers  # seconds per whole decode step
+
+    def describe(self, reps):
+        w = self.w
+        return (f"{reps} sampled decode tokens, each for {self.B} queries of one layer: route "
+                f"against {self.nd} of {self.n_docs} documents, top-{w.top_k} over all "
+                f"{self.n_docs}, attention over {w.top_k} docs + {w.query_tokens + 1} local rows; "
+                f"scaled linearly to {w.batch} queries x {w.n_layers} layers x {self.n_docs} "
+                f"documents (extrapolated)")
+
+
+def cpu_baseline(w, seed=1234, budget_s=12.0):
+    t_start = time.perf_counter()
+    smp = OracleSample(w, seed, n_docs_sample=128, queries=2)
+    times = []
+    t0 = time.perf_counter()
+    while not times or time.perf_counter() - t0 < budget_s:
+        times.append(smp.step())
+    step_s = statistics.median(times)
+    return {"value": round(1.0 / step_s, 6), "unit": "steps/s", "cores": smp.cores,
+            "kind": "oracle", "sample": smp.describe(len(times)),
+            "seconds": round(time.perf_counter() - t_start, 1)}
+
+
+def run_reference(args, w):
+    K, Wm = args.steps, args.warmup
+    smp = OracleSample(w, 1234, n_docs_sample=32, queries=1)
+    vals = []
+    t_all = time.perf_counter()
+    for i in range(Wm + K):
+        v = smp.step()
+        if i >= Wm:
+            vals.append(v)
+        if time.perf_counter() - t_all > 240:
+            break
+    value = round(1.0 / statistics.median(vals), 6)
+    return {
+        "metric": METRIC, "impl": "reference", "value": value,
+        "unit": "steps/s", "n_gpus": 1, "steps": len(vals), "warmup": Wm,
+        "ms_per_step": round(1e3 / value, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "layers": w.n_layers, "batch": w.batch, "top_k": w.top_k},
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": smp.cores, "kind": "oracle",
+                         "sample": smp.describe(len(vals))},
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, w)))
+        return
+    world, rank, local = dist_setup(args)
+    res = run_gpu(args, w, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(res))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -24,40 +24,66 @@ constexpr int kMaxMemRows = 4096;  // retrieved chunks per query (k * chunks per
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Chunk list of query b's retrieved documents in rank order -> table[0..n_mem).
+// Warp 0 loads the k (<= 64) ranks' chunk counts in parallel (two ranks per
+// lane) and prefix-sums them with shuffles; every thread then fills table
+// entries from shared memory only (binary search over the prefix sums).
 // Ids outside [0, n_docs) contribute no rows and raise MSA_DEVERR_BAD_DOC_ID.
-// slot_of_rank (nullable, [B][k]): chunk rows of rank r start at
-// slot_of_rank[b][r] * slot_chunks instead of doc_chunk_off[id].
+// slots_b (nullable, [k]): chunk rows of rank r start at slots_b[r] *
+// slot_chunks instead of doc_chunk_off[id] (device slot cache of a host tier).
+// `pre` needs kMaxTopK + 1 ints and `base` kMaxTopK ints of shared memory.
 __device__ __forceinline__ int build_chunk_table(const int32_t *__restrict__ ids_b, int k,
                                                  const int64_t *__restrict__ doc_chunk_off,
                                                  int n_docs, const int32_t *__restrict__ slots_b,
                                                  int slot_chunks, int *table, int *pre,
-                                                 int table_cap) {
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int r = 0; r < k; ++r) {
-      pre[r] = acc;
-      const int d = ids_b[r];
-      int cnt = 0;
-      if (d >= 0 && d < n_docs) {
-        cnt = static_cast<int>(doc_chunk_off[d + 1] - doc_chunk_off[d]);
-      } else {
-        raise_device_error(MSA_DEVERR_BAD_DOC_ID);
+                                                 int *base, int table_cap) {
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int cnt[2] = {0, 0};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = lane + 32 * h;
+      if (r < k) {
+        const int d = ids_b[r];
+        if (d >= 0 && d < n_docs) {
+          const int64_t c0 = doc_chunk_off[d];
+          cnt[h] = static_cast<int>(doc_chunk_off[d + 1] - c0);
+          base[r] = slots_b ? slots_b[r] * slot_chunks : static_cast<int>(c0);
+        } else {
+          raise_device_error(MSA_DEVERR_BAD_DOC_ID);
+          base[r] = 0;
+        }
       }
-      if (acc + cnt > table_cap) cnt = 0;  // host validation keeps this unreachable
-      acc += cnt;
     }
-    pre[k] = acc;
+    int run = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      int v = cnt[h];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      const int r = lane + 32 * h;
+      const int excl = run + v - cnt[h];
+      // a rank that would overflow the table contributes nothing (host validation keeps
+      // k * max_doc_chunks <= table_cap, so this does not happen)
+      if (r < k) pre[r] = excl + cnt[h] > table_cap ? min(excl, table_cap) : excl;
+      run += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) pre[k] = min(run, table_cap);
   }
   __syncthreads();
-  for (int r = 0; r < k; ++r) {
-    const int cnt = pre[r + 1] - pre[r];
-    if (cnt == 0) continue;
-    const int d = ids_b[r];
-    const int64_t base = slots_b ? static_cast<int64_t>(slots_b[r]) * slot_chunks : doc_chunk_off[d];
-    for (int jj = threadIdx.x; jj < cnt; jj += blockDim.x) table[pre[r] + jj] = static_cast<int>(base + jj);
+  const int n_mem = pre[k];
+  for (int x = threadIdx.x; x < n_mem; x += blockDim.x) {
+    int lo = 0, hi = k - 1;  // last rank r with pre[r] <= x
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    table[x] = base[lo] + (x - pre[lo]);
   }
   __syncthreads();
-  return pre[k];
+  return n_mem;
 }
 
 // ---------------------------------------------------------------- append
@@ -116,11 +142,12 @@ attend_simt_kernel(const T *__restrict__ content, const int32_t *__restrict__ id
   constexpr int U = D / 32;
   __shared__ int table[kMaxMemRows];
   __shared__ int pre[kMaxTopK + 1];
+  __shared__ int base[kMaxTopK];
   const int b = blockIdx.x / T_tok, i = blockIdx.x % T_tok;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_mem = build_chunk_table(ids + static_cast<int64_t>(b) * k, k, doc_chunk_off, n_docs,
                                       slots ? slots + static_cast<int64_t>(b) * k : nullptr,
-                                      slot_chunks, table, pre, kMaxMemRows);
+                                      slot_chunks, table, pre, base, kMaxMemRows);
   const int j = cache_len[b] + i;
   const int h = warp;
   if (h >= H_q) return;
@@ -189,7 +216,7 @@ struct AttSmem {
   static constexpr int kMergeBytes = kAttWarps * 16 * (D + 2) * 4;
   static constexpr int kRing = kAttWarps * kWarpBytes;
   static constexpr int kFixed =
-      (kRing > kMergeBytes ? kRing : kMergeBytes) + kQBytes + (kMaxTopK + 1) * 4;
+      (kRing > kMergeBytes ? kRing : kMergeBytes) + kQBytes + (2 * kMaxTopK + 1) * 4;
   static int bytes(int table_cap) { return kFixed + table_cap * 4; }
 };
 
@@ -218,7 +245,8 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
   uint8_t *ring = sm;
   uint8_t *qsm = sm + (Sm::kRing > Sm::kMergeBytes ? Sm::kRing : Sm::kMergeBytes);
   int *pre = reinterpret_cast<int *>(qsm + Sm::kQBytes);
-  int *table = pre + (kMaxTopK + 1);
+  int *base = pre + (kMaxTopK + 1);
+  int *table = base + kMaxTopK;
 
   const int H_q = H_kv * G;
   const int b = blockIdx.x / H_kv, g = blockIdx.x % H_kv;
@@ -227,7 +255,7 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
 
   const int n_mem = build_chunk_table(ids + static_cast<int64_t>(b) * k, k, doc_chunk_off, n_docs,
                                       slots ? slots + static_cast<int64_t>(b) * k : nullptr,
-                                      slot_chunks, table, pre, table_cap);
+                                      slot_chunks, table, pre, base, table_cap);
   const int j = cache_len[b] + i;
   const bool overflow = j >= cap;
   const int n_ctx = overflow ? 0 : n_mem + j + 1;
