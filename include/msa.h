@@ -219,6 +219,38 @@ MSA_API msa_status msa_sparse_attend(const msa_memory *mem, const void *content,
                              void *O, void *workspace, size_t workspace_bytes,
                              msa_stream stream);
 
+/*
+ * msa_sparse_attend_static -- the same attention as msa_sparse_attend, for
+ * callers that cannot allocate device memory: for example a plugin inside a
+ * host engine that reserved the whole device memory budget up front and
+ * forbids any further allocation, or a C caller with no allocator of its own
+ * to size a workspace.  The pages have no counterpart to this call; it is an
+ * engineering entry point of this library.
+ *
+ * Arguments are those of msa_sparse_attend without `workspace` and
+ * `workspace_bytes`; the caller still passes every input and output buffer.
+ * The call allocates nothing.  Its scratch (the partial results of the split
+ * attention context) lives in one fixed device array of 8 MiB (8388608 bytes)
+ * inside the library; every GPU that loads the library holds that array until
+ * the process exits.  A call whose scratch would exceed 8 MiB (the size
+ * msa_attend_workspace_size reports for the same arguments, with
+ * cache_capacity in place of max_local_position) is rejected with
+ * MSA_ERR_UNSUPPORTED and enqueues nothing.
+ *
+ * The first call on a device looks up that device's address of the array
+ * (cudaGetSymbolAddress, with the device current); make that first call before
+ * any stream capture.  All calls share the one array and each call overwrites
+ * it: calls that may run at the same time on the GPU (different streams, or
+ * different host threads) race and must be ordered by the caller.  Nothing in
+ * the array needs clearing: every scratch entry a call reads was written by
+ * the same call.
+ */
+MSA_API msa_status msa_sparse_attend_static(
+    const msa_memory *mem, const void *content, const int32_t *ids, int32_t batch,
+    int32_t k, int32_t tokens, int32_t n_q_heads, const void *Q, const void *K_new,
+    const void *V_new, void *K_cache, void *V_cache, int32_t *cache_len,
+    int32_t cache_capacity, int32_t pos_offset, void *O, msa_stream stream);
+
 /* Per-layer decode state, every buffer owned by the caller (see msa_step). */
 typedef struct {
   int32_t batch;

@@ -15,6 +15,12 @@
 #include "route.cuh"
 #include "topk.cuh"
 
+// Scratch of msa_sparse_attend_static: a fixed device array, so that callers
+// which cannot allocate device memory still get the split-context attention.
+// Every GPU that loads the library holds these 8 MiB until the process exits.
+static constexpr size_t kStaticAttendScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) uint8_t g_attend_static_scratch[kStaticAttendScratchBytes];
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -44,6 +50,26 @@ msa_status cuda_fail(cudaError_t e, const char *what) {
     cudaError_t e_ = cudaGetLastError();                \
     if (e_ != cudaSuccess) return cuda_fail(e_, what);  \
   } while (0)
+
+// Device address of the static attention scratch on the current device, looked
+// up once per device (cudaGetSymbolAddress with that device current).
+msa_status static_attend_scratch(void **out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void *addr[kMaxDevices] = {};
+  int dev = 0;
+  MSA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(MSA_ERR_UNSUPPORTED, "device %d", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_attend_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static attention scratch)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return MSA_OK;
+}
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -609,6 +635,29 @@ msa_status msa_sparse_attend(const msa_memory *mem, const void *content, const i
   return attend_impl(mem, content, ids, nullptr, 0, batch, k, tokens, n_q_heads, Q, K_new, V_new,
                      K_cache, V_cache, cache_len, cache_capacity, pos_offset, O, workspace,
                      workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+msa_status msa_sparse_attend_static(const msa_memory *mem, const void *content,
+                                    const int32_t *ids, int32_t batch, int32_t k, int32_t tokens,
+                                    int32_t n_q_heads, const void *Q, const void *K_new,
+                                    const void *V_new, void *K_cache, void *V_cache,
+                                    int32_t *cache_len, int32_t cache_capacity,
+                                    int32_t pos_offset, void *O, msa_stream stream) {
+  if (!mem) return fail(MSA_ERR_INVALID_ARG, "null memory");
+  if (batch < 1 || tokens < 1 || k < 0 || k > msa::kMaxTopK || n_q_heads < 1 ||
+      cache_capacity < 1)
+    return fail(MSA_ERR_INVALID_ARG, "bad batch, tokens, k, n_q_heads or cache_capacity");
+  const AttendPlan plan = plan_attend(mem, batch, tokens, k, n_q_heads, cache_capacity);
+  if (plan.bytes > kStaticAttendScratchBytes)
+    return fail(MSA_ERR_UNSUPPORTED,
+                "this call needs %zu bytes of attention scratch; the static scratch holds %zu",
+                plan.bytes, kStaticAttendScratchBytes);
+  void *scratch = nullptr;
+  const msa_status s = static_attend_scratch(&scratch);
+  if (s != MSA_OK) return s;
+  return attend_impl(mem, content, ids, nullptr, 0, batch, k, tokens, n_q_heads, Q, K_new, V_new,
+                     K_cache, V_cache, cache_len, cache_capacity, pos_offset, O, scratch,
+                     kStaticAttendScratchBytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t msa_step_workspace_size(const msa_memory *mem, int32_t batch, int32_t k, int32_t n_q_heads) {

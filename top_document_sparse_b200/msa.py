@@ -73,6 +73,8 @@ SIGNATURES = {
     "msa_attend_workspace_size": (_SZ, [_P, _I32, _I32, _I32, _I32]),
     "msa_sparse_attend": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P,
                                          _P, _I32, _I32, _P, _P, _SZ, _P]),
+    "msa_sparse_attend_static": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P,
+                                                _P, _P, _P, _I32, _I32, _P, _P]),
     "msa_step_workspace_size": (_SZ, [_P, _I32, _I32, _I32]),
     "msa_step": (ctypes.c_int, [_P, _P, _P, ctypes.POINTER(DecodeState), _P, _P, _P, _P, _P, _P]),
     "msa_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
@@ -215,6 +217,16 @@ class Memory:
                                       _ptr(K_new), _ptr(V_new), _ptr(K_cache), _ptr(V_cache),
                                       _ptr(cache_len), K_cache.shape[1], pos_offset, _ptr(O),
                                       _ptr(workspace), ws_bytes, _stream(stream)))
+
+    def sparse_attend_static(self, content, ids, Q, K_new, V_new, K_cache, V_cache, cache_len,
+                             pos_offset: int, O, stream=None):
+        """msa_sparse_attend without a workspace: scratch from the library's fixed array."""
+        B, T, H_q, _ = Q.shape
+        k = ids.shape[1] if ids is not None else 0
+        _check(_lib.msa_sparse_attend_static(self.handle, _ptr(content), _ptr(ids), B, k, T, H_q,
+                                             _ptr(Q), _ptr(K_new), _ptr(V_new), _ptr(K_cache),
+                                             _ptr(V_cache), _ptr(cache_len), K_cache.shape[1],
+                                             pos_offset, _ptr(O), _stream(stream)))
 
     def step_workspace_size(self, batch: int, k: int, n_q_heads: int) -> int:
         return _lib.msa_step_workspace_size(self.handle, batch, k, n_q_heads)
