@@ -264,6 +264,39 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
   const int x0 = split * per;
   const int x1 = min(n_ctx, x0 + per);
 
+  const int64_t kv = static_cast<int64_t>(H_kv) * D;
+  uint8_t *wbuf = ring + warp * Sm::kWarpBytes;
+  // issue the loads of the block starting at context row x into stage s
+  auto issue = [&](int x, int s) {
+    uint8_t *kb = wbuf + s * 2 * Sm::kBlockBytes;
+    uint8_t *vb = kb + Sm::kBlockBytes;
+#pragma unroll
+    for (int u = 0; u < kAttRows * CPR / 32; ++u) {
+      const int idx = lane + 32 * u;
+      const int r = idx / CPR, c = idx % CPR;
+      const int xr = x + r;
+      const __nv_bfloat16 *ks = K_cache, *vs = V_cache;
+      bool ok = xr < x1;
+      if (ok) {
+        if (xr < n_mem) {
+          ks = content + static_cast<int64_t>(table[xr]) * 2 * kv + g * D;
+          vs = ks + kv;
+        } else {
+          const int64_t row = (static_cast<int64_t>(b) * cap + (xr - n_mem)) * kv + g * D;
+          ks = K_cache + row;
+          vs = V_cache + row;
+        }
+      }
+      cp_async_16(smem_u32(kb + swz<D>(r, c)), ks + c * 8, ok);
+      cp_async_16(smem_u32(vb + swz<D>(r, c)), vs + c * 8, ok);
+    }
+    cp_async_commit();
+  };
+
+  // the first context block is in flight while the query is rotated
+  const int nblk = (x1 > x0) ? (x1 - x0 + kAttRows - 1) / kAttRows : 0;
+  int s = 0;
+  if (warp < nblk) issue(x0 + warp * kAttRows, 0);
   // rotated query rows of the group -> qsm [16][D] (rows >= G are zero)
   {
     const int half = D / 2;
@@ -297,35 +330,6 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
     }
   }
 
-  const int64_t kv = static_cast<int64_t>(H_kv) * D;
-  uint8_t *wbuf = ring + warp * Sm::kWarpBytes;
-  // issue the loads of the block starting at context row x into stage s
-  auto issue = [&](int x, int s) {
-    uint8_t *kb = wbuf + s * 2 * Sm::kBlockBytes;
-    uint8_t *vb = kb + Sm::kBlockBytes;
-#pragma unroll
-    for (int u = 0; u < kAttRows * CPR / 32; ++u) {
-      const int idx = lane + 32 * u;
-      const int r = idx / CPR, c = idx % CPR;
-      const int xr = x + r;
-      const __nv_bfloat16 *ks = K_cache, *vs = V_cache;
-      bool ok = xr < x1;
-      if (ok) {
-        if (xr < n_mem) {
-          ks = content + static_cast<int64_t>(table[xr]) * 2 * kv + g * D;
-          vs = ks + kv;
-        } else {
-          const int64_t row = (static_cast<int64_t>(b) * cap + (xr - n_mem)) * kv + g * D;
-          ks = K_cache + row;
-          vs = V_cache + row;
-        }
-      }
-      cp_async_16(smem_u32(kb + swz<D>(r, c)), ks + c * 8, ok);
-      cp_async_16(smem_u32(vb + swz<D>(r, c)), vs + c * 8, ok);
-    }
-    cp_async_commit();
-  };
-
   float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 domain) of rows g8 and g8+8
   float l0 = 0.0f, l1 = 0.0f;
   float acc[D / 8][4];
@@ -334,9 +338,6 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[n][e] = 0.0f;
 
-  const int nblk = (x1 > x0) ? (x1 - x0 + kAttRows - 1) / kAttRows : 0;
-  int s = 0;
-  if (warp < nblk) issue(x0 + warp * kAttRows, 0);
   for (int bi = warp; bi < nblk; bi += kAttWarps) {
     const int x = x0 + bi * kAttRows;
     if (bi + kAttWarps < nblk) {

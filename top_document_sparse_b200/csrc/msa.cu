@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "pool.cuh"
 #include "route.cuh"
+#include "route_tc.cuh"
 #include "topk.cuh"
 
 // Scratch of msa_sparse_attend_static: a fixed device array, so that callers
@@ -184,31 +185,32 @@ RoutePlan plan_route(const msa_memory *mem, int B, int T, int k) {
 }
 
 template <int NT>
-msa_status launch_route_mma(const msa_memory *mem, const void *keys, const void *qhat, int R,
-                            int T, float *state, cudaStream_t st) {
+msa_status launch_route_tc(const msa_memory *mem, const void *keys, const void *qhat, int R, int T,
+                           float *state, cudaStream_t st) {
+  using L = msa::RouteTcLayout<NT>;
   const int W = mem->H_r * mem->d_r;
   CUtensorMap tmK, tmQ;
-  msa_status s = make_map_bf16(&tmK, keys, mem->n_chunks, W, msa::kRouteTileC);
+  msa_status s = make_map_bf16(&tmK, keys, mem->n_chunks, W, L::kTileC);
   if (s != MSA_OK) return s;
   s = make_map_bf16(&tmQ, qhat, R, W, NT);
   if (s != MSA_OK) return s;
   const int maxs = max_dyn_smem();
-  int stages = 8;
-  while (stages > 2 && msa::RouteLayout<NT>::bytes(W, stages) > static_cast<size_t>(maxs)) --stages;
-  const size_t smem = msa::RouteLayout<NT>::bytes(W, stages);
-  if (smem > static_cast<size_t>(maxs))
+  int stages = 12;  // (256 B left for the epilogue's static shared memory)
+  while (stages > 2 && L::bytes(W, stages) + 256 > static_cast<size_t>(maxs)) --stages;
+  const size_t smem = L::bytes(W, stages);
+  if (smem + 256 > static_cast<size_t>(maxs))
     return fail(MSA_ERR_UNSUPPORTED, "router width %d needs %zu B of shared memory", W, smem);
-  auto kern = msa::route_mma_kernel<NT>;
+  auto kern = msa::route_tc_kernel<NT>;
   MSA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  const int n_ct = static_cast<int>((mem->n_chunks + msa::kRouteTileC - 1) / msa::kRouteTileC);
+  const int n_ct = static_cast<int>((mem->n_chunks + L::kTileC - 1) / L::kTileC);
   const int n_rt = (R + NT - 1) / NT;
   const int64_t n_tiles = static_cast<int64_t>(n_ct) * n_rt;
   if (n_tiles > INT32_MAX) return fail(MSA_ERR_UNSUPPORTED, "too many route tiles");
   const int grid = static_cast<int>(std::min<int64_t>(n_tiles, num_sms()));
-  kern<<<grid, 160, smem, st>>>(tmK, tmQ, mem->n_chunks, R, W, T, 1.0f / mem->H_r,
+  kern<<<grid, 192, smem, st>>>(tmK, tmQ, mem->n_chunks, R, W, T, 1.0f / mem->H_r,
                                 mem->d_chunk_doc, mem->n_docs, state, n_ct,
                                 static_cast<int>(n_tiles), stages);
-  MSA_LAUNCHED("route_mma_kernel");
+  MSA_LAUNCHED("route_tc_kernel");
   return MSA_OK;
 }
 
@@ -244,11 +246,11 @@ msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, i
       MSA_LAUNCHED("qnorm_kernel");
       msa_status s;
       if (R <= 16)
-        s = launch_route_mma<16>(mem, keys, qh, R, T, state, st);
+        s = launch_route_tc<16>(mem, keys, qh, R, T, state, st);
       else if (R <= 32)
-        s = launch_route_mma<32>(mem, keys, qh, R, T, state, st);
+        s = launch_route_tc<32>(mem, keys, qh, R, T, state, st);
       else
-        s = launch_route_mma<64>(mem, keys, qh, R, T, state, st);
+        s = launch_route_tc<64>(mem, keys, qh, R, T, state, st);
       if (s != MSA_OK) return s;
     } else {
       auto *qh = reinterpret_cast<float *>(wsb + plan.qhat);

@@ -59,19 +59,65 @@ __device__ __forceinline__ void epi_token_max(float *S, int ldS, int MC, int NR,
   }
 }
 
-// Stage 2: for each (document run inside the tile, query), max over the run's
-// chunks, then atomic max into state.
+// Stage 2 (all nthr threads must call it: it holds named barrier 2): for each
+// (document run inside the tile, query), max over the run's
+// chunks, then max-merge into state.  `segs` (shared, >= MC + 1 ints) receives
+// the run starts.  A run whose document lies wholly inside the chunk tile, for
+// a query whose rows lie wholly inside the row tile, has this CTA as its only
+// writer during the call: it is merged with a plain load / max / store
+// (consecutive threads take consecutive documents, so the accesses coalesce).
+// Runs of documents that straddle a tile edge, and queries split over row
+// tiles, use an atomic float max.
+//   prev_doc / next_doc: document of the chunk just before / after the tile
+//   (-1 at the memory's ends); q_lo / q_hi: the queries whose rows are all
+//   inside the row tile are [q_lo, q_hi) (relative to b0).
 __device__ __forceinline__ void epi_doc_max(const float *S, int ldS, int MC, int QB, int64_t b0,
-                                            const int *docs, int n_docs, float *state, int tid,
-                                            int nthr) {
-  for (int p = tid; p < MC * QB; p += nthr) {
-    const int q = p / MC, m = p % MC;
-    const int d = docs[m];
-    if (m > 0 && docs[m - 1] == d) continue;
-    float v = S[m * ldS + q];
-    for (int m2 = m + 1; m2 < MC && docs[m2] == d; ++m2) v = fmaxf(v, S[m2 * ldS + q]);
-    atomic_max_float(state + (b0 + q) * n_docs + d, v);
+                                            const int *docs, int prev_doc, int next_doc,
+                                            int q_lo, int q_hi, int n_docs, float *state,
+                                            int *segs, int tid, int nthr, bool write = true) {
+  // run starts by a block-wide ordered compaction (nthr == 128: four warps)
+  const int lane = tid & 31, warp = tid >> 5;
+  __shared__ int warp_cnt[8];
+  int n_seg = 0;
+  for (int base = 0; base < MC; base += nthr) {
+    const int m = base + tid;
+    const bool start = m < MC && (m == 0 || docs[m] != docs[m - 1]);
+    const unsigned bal = __ballot_sync(0xffffffffu, start);
+    if (lane == 0) warp_cnt[warp] = __popc(bal);
+    asm volatile("bar.sync 2, %0;" ::"r"(nthr) : "memory");
+    int before = n_seg;
+    for (int w = 0; w < warp; ++w) before += warp_cnt[w];
+    if (start) segs[before + __popc(bal & ((1u << lane) - 1))] = m;
+    for (int w = 0; w < nthr / 32; ++w) n_seg += warp_cnt[w];
+    asm volatile("bar.sync 2, %0;" ::"r"(nthr) : "memory");
   }
+  if (tid == 0) segs[n_seg] = MC;
+  asm volatile("bar.sync 2, %0;" ::"r"(nthr) : "memory");
+  if (!write) return;  // every thread has passed the barriers above
+  for (int p = tid; p < n_seg * QB; p += nthr) {
+    const int q = p / n_seg, g = p - q * n_seg;
+    const int m0 = segs[g], m1 = segs[g + 1];
+    const int d = docs[m0];
+    float v = S[m0 * ldS + q];
+    for (int m = m0 + 1; m < m1; ++m) v = fmaxf(v, S[m * ldS + q]);
+    float *dst = state + (b0 + q) * n_docs + d;
+    const bool whole_doc = (m0 > 0 || prev_doc != d) && (m1 < MC || next_doc != d);
+    if (whole_doc && q >= q_lo && q < q_hi) {
+      *dst = fmaxf(*dst, v);
+    } else {
+      atomic_max_float(dst, v);
+    }
+  }
+}
+
+// Queries (relative to b0 = r0 / T) whose T rows all lie in [r0, r0 + NR).
+__device__ __forceinline__ void query_span(int64_t r0, int NR, int T_tok, int64_t b0, int &q_lo,
+                                           int &q_hi) {
+  const int64_t first_full = (r0 + T_tok - 1) / T_tok;  // first query starting at or after r0
+  const int64_t end_full = (r0 + NR) / T_tok;           // queries ending at or before r0 + NR
+  q_lo = static_cast<int>(first_full - b0);
+  q_hi = static_cast<int>(end_full - b0);
+  if (q_hi < q_lo) q_hi = q_lo;
 }
 
 // ---------------------------------------------------------------- fp32 path
@@ -86,6 +132,7 @@ route_simt_kernel(const T *__restrict__ Khat, const T *__restrict__ Qhat, int64_
   __shared__ float Qs[32][33];
   __shared__ float S[32 * 33];
   __shared__ int docs[32];
+  __shared__ int segs[33];
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 32;
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 32;
   const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
@@ -113,196 +160,17 @@ route_simt_kernel(const T *__restrict__ Khat, const T *__restrict__ Qhat, int64_
 #pragma unroll
     for (int b = 0; b < 2; ++b) S[(ty + 16 * a) * 33 + tx + 16 * b] = acc[a][b] * inv_Hr;
   if (tid < MC) docs[tid] = chunk_doc[c0 + tid];
+  const int prev_doc = c0 > 0 ? chunk_doc[c0 - 1] : -1;
+  const int next_doc = c0 + MC < C ? chunk_doc[c0 + MC] : -1;
   __syncthreads();
   epi_token_max(S, 33, MC, NR, r0, T_tok, tid, 256);
   __syncthreads();
   const int64_t b0 = r0 / T_tok;
   const int QB = static_cast<int>((r0 + NR - 1) / T_tok - b0 + 1);
-  epi_doc_max(S, 33, MC, QB, b0, docs, n_docs, state, tid, 256);
-}
-
-// ---------------------------------------------------------------- bf16 path
-// Tensor-core route.  A CTA is a persistent loop over (row tile, chunk tile)
-// pairs; a chunk tile is 128 chunks, a row tile NT query rows.  Warp 4 is the
-// producer: one lane issues TMA loads of 64-feature slices (128 rows x 128 B,
-// 128B-swizzled) of the unit router keys into a ring of `stages` buffers, and
-// of the normalised query rows (all W features of NT rows, resident while the
-// row tile lasts).  Warps 0-3 each own 32 chunks of the tile and run
-// mma.sync m16n8k16 (bf16 in, fp32 accumulate) over the slices, then the
-// shared epilogue.  Every barrier wait is bounded.
-constexpr int kRouteTileC = 128;
-constexpr int kRouteSliceBytes = kRouteTileC * 128;  // 16 KiB
-
-template <int NT>
-struct RouteLayout {
-  static __host__ __device__ size_t q_bytes(int W) { return static_cast<size_t>(W / 64) * NT * 128; }
-  static __host__ __device__ size_t s_bytes() { return static_cast<size_t>(kRouteTileC) * (NT + 1) * 4; }
-  static __host__ __device__ size_t bytes(int W, int stages) {
-    return 1024 /*alignment slack*/ + q_bytes(W) + static_cast<size_t>(stages) * kRouteSliceBytes +
-           s_bytes() + kRouteTileC * 4 + (2 * stages + 2) * 8 + 16;
-  }
-};
-
-template <int NT>
-__global__ void __launch_bounds__(160, 1)
-route_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-                 int64_t C, int R, int W, int T_tok, float inv_Hr,
-                 const int32_t *__restrict__ chunk_doc, int n_docs, float *__restrict__ state,
-                 int n_chunk_tiles, int n_tiles, int stages) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int KS = W / 64;
-  uint8_t *Qs = smem;
-  uint8_t *Ks = Qs + RouteLayout<NT>::q_bytes(W);
-  float *Sb = reinterpret_cast<float *>(Ks + static_cast<size_t>(stages) * kRouteSliceBytes);
-  int *docs = reinterpret_cast<int *>(Sb + kRouteTileC * (NT + 1));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(docs + kRouteTileC);
-  // written only by consumer warps, read only after a consumer barrier, so
-  // every consumer warp takes the same abort decision
-  volatile int *cons_abort = reinterpret_cast<volatile int *>(bars + 2 * stages + 2);
-  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + stages);
-  const uint32_t qfull = smem_u32(bars + 2 * stages), qempty = smem_u32(bars + 2 * stages + 1);
-  const uint32_t qs_addr = smem_u32(Qs), ks_addr = smem_u32(Ks);
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  constexpr int LD = NT + 1;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 4);
-    }
-    mbar_init(qfull, 1);
-    mbar_init(qempty, 4);
-    *cons_abort = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  if (warp == 4) {  // ------------------------------------------- producer
-    if (lane != 0) return;
-    prefetch_tensormap(&tmK);
-    prefetch_tensormap(&tmQ);
-    const uint64_t pol = policy_evict_first();
-    int it = 0, qloads = 0, cur_rt = -1;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-      const int rt = tile / n_chunk_tiles, ct = tile % n_chunk_tiles;
-      if (rt != cur_rt) {
-        if (qloads > 0 && !mbar_wait(qempty, (qloads - 1) & 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(qfull, static_cast<uint32_t>(KS * NT * 128));
-        for (int s = 0; s < KS; ++s) tma_load_2d(qs_addr + s * NT * 128, &tmQ, 64 * s, rt * NT, qfull);
-        ++qloads;
-        cur_rt = rt;
-      }
-      for (int s = 0; s < KS; ++s) {
-        const int st = it % stages;
-        if (it >= stages && !mbar_wait(empty0 + 8 * st, ((it / stages) - 1) & 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(full0 + 8 * st, kRouteSliceBytes);
-        tma_load_2d_hint(ks_addr + st * kRouteSliceBytes, &tmK, 64 * s, ct * kRouteTileC,
-                         full0 + 8 * st, pol);
-        ++it;
-      }
-    }
-    if (!ok) {
-      raise_device_error(MSA_DEVERR_WAIT_TIMEOUT);
-      // let every copy this thread issued land before the CTA can exit
-      for (int j = (it > stages ? it - stages : 0); j < it; ++j)
-        mbar_wait(full0 + 8 * (j % stages), (j / stages) & 1);
-      if (qloads > 0) mbar_wait(qfull, (qloads - 1) & 1);
-    }
-    return;
-  }
-
-  // ----------------------------------------------------------- consumers
-  const int tid = threadIdx.x;  // 0..127
-  int it = 0, quses = 0, cur_rt = -1;
-  bool failed = false;
-  for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-    const int rt = tile / n_chunk_tiles, ct = tile % n_chunk_tiles;
-    if (rt != cur_rt) {
-      if (quses > 0) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(qempty);
-      }
-      if (!failed && !mbar_wait(qfull, quses & 1)) failed = true;
-      ++quses;
-      cur_rt = rt;
-    }
-    float acc[2][NT / 8][4];
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int n = 0; n < NT / 8; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[a][n][e] = 0.0f;
-
-    for (int s = 0; s < KS; ++s, ++it) {
-      const int st = it % stages;
-      if (!failed && !mbar_wait(full0 + 8 * st, (it / stages) & 1)) failed = true;
-      if (!failed) {
-        const uint32_t kbase = ks_addr + st * kRouteSliceBytes;
-        const uint32_t qbase = qs_addr + s * NT * 128;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          uint32_t a[2][4];
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            const int row = warp * 32 + mt * 16 + (lane & 15);
-            const int chunk = 2 * kk + (lane >> 4);
-            ldsm_x4(kbase + row * 128 + ((chunk ^ (row & 7)) << 4), a[mt][0], a[mt][1], a[mt][2],
-                    a[mt][3]);
-          }
-#pragma unroll
-          for (int ng = 0; ng < NT / 16; ++ng) {
-            const int row = ng * 16 + (lane & 7) + ((lane >> 4) << 3);
-            const int chunk = 2 * kk + ((lane >> 3) & 1);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(qbase + row * 128 + ((chunk ^ (row & 7)) << 4), b0, b1, b2, b3);
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-              mma_bf16_16816(acc[mt][2 * ng], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
-              mma_bf16_16816(acc[mt][2 * ng + 1], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b2, b3);
-            }
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8 * st);
-    }
-    if (failed) *cons_abort = 1;
-
-    // epilogue: scores -> shared, token max, document max -> state
-    const int64_t c0 = static_cast<int64_t>(ct) * kRouteTileC;
-    const int64_t r0 = static_cast<int64_t>(rt) * NT;
-    const int MC = static_cast<int>(C - c0 < kRouteTileC ? C - c0 : kRouteTileC);
-    const int NR = static_cast<int>(R - r0 < NT ? R - r0 : NT);
-    {
-      const int g = lane >> 2, q2 = (lane & 3) * 2;
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int n = 0; n < NT / 8; ++n) {
-          const int m = warp * 32 + mt * 16 + g;
-          const int col = n * 8 + q2;
-          Sb[m * LD + col] = acc[mt][n][0] * inv_Hr;
-          Sb[m * LD + col + 1] = acc[mt][n][1] * inv_Hr;
-          Sb[(m + 8) * LD + col] = acc[mt][n][2] * inv_Hr;
-          Sb[(m + 8) * LD + col + 1] = acc[mt][n][3] * inv_Hr;
-        }
-    }
-    if (tid < MC) docs[tid] = chunk_doc[c0 + tid];
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    const bool abort_now = *cons_abort != 0;
-    if (!abort_now) epi_token_max(Sb, LD, MC, NR, r0, T_tok, tid, 128);
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    const int64_t b0 = r0 / T_tok;
-    const int QB = static_cast<int>((r0 + NR - 1) / T_tok - b0 + 1);
-    if (!abort_now) epi_doc_max(Sb, LD, MC, QB, b0, docs, n_docs, state, tid, 128);
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (abort_now) break;
-  }
-  if (failed) raise_device_error(MSA_DEVERR_WAIT_TIMEOUT);
+  int q_lo, q_hi;
+  query_span(r0, NR, T_tok, b0, q_lo, q_hi);
+  epi_doc_max(S, 33, MC, QB, b0, docs, prev_doc, next_doc, q_lo, q_hi, n_docs, state, segs, tid,
+              256);
 }
 
 }  // namespace msa

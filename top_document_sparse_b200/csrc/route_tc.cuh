@@ -1,0 +1,223 @@
+// route_tc.cuh -- tensor-core (tcgen05) route score for bf16 memories
+// (MSA, b-lab.team summary item 1 "Scalable Sparse Attention"; stage "Online
+// Routing & Context Assembly").
+//
+// s[c, r] = (1/H_r) * <Khat[c], Qhat[r]> over W = H_r * d_r features, with
+// Khat the unit router keys (per head) and Qhat the normalised query rows, so
+// s is the mean over router heads of the per-head cosines.  A tile is 128
+// chunks (UMMA M) x NT query rows (UMMA N); D lives in TMEM.
+//
+// Warp roles (192 threads):
+//   warp 4  one lane: TMA producer -- query rows of the row tile (resident,
+//           all W features) and a ring of 64-feature x 128-chunk key slices
+//   warp 5  allocates TMEM; one lane issues 4 UMMAs (K = 16 each) per slice
+//           and commits them to the slice's "empty" barrier, then commits
+//           the finished accumulator to "acc full"
+//   warps 0-3  epilogue: thread t drains TMEM lane t (chunk t of the tile),
+//           scales, then the shared token-max / document-max epilogue with
+//           an atomic max into the running state
+// Two TMEM accumulators alternate, so the epilogue of tile i overlaps the MMAs
+// of tile i+1.  Every barrier wait is bounded; a wait that runs out raises
+// MSA_DEVERR_WAIT_TIMEOUT, later waits are skipped, in-flight copies and MMAs
+// are drained, and TMEM is freed before the CTA exits.
+#pragma once
+#include "route.cuh"
+#include "tc05.cuh"
+
+namespace msa {
+
+template <int NT>
+struct RouteTcLayout {
+  static constexpr int kTileC = 128;
+  static constexpr int kSlice = kTileC * 128;  // 16 KiB: 128 rows x 64 bf16
+  static constexpr int kLD = NT + 1;           // epilogue staging row stride (floats)
+  static constexpr uint32_t kTmemCols = (2 * NT < 32) ? 32 : 2 * NT;
+  static __host__ __device__ size_t q_bytes(int W) { return static_cast<size_t>(W / 64) * NT * 128; }
+  static __host__ __device__ size_t bytes(int W, int stages) {
+    return 1024 + q_bytes(W) + static_cast<size_t>(stages) * kSlice +
+           static_cast<size_t>(kTileC) * kLD * 4 + (2 * kTileC + 8) * 4 + (2 * stages + 7) * 8 +
+           32;
+  }
+};
+
+template <int NT>
+__global__ void __launch_bounds__(192, 1)
+route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
+                int64_t C, int R, int W, int T_tok, float inv_Hr,
+                const int32_t *__restrict__ chunk_doc, int n_docs, float *__restrict__ state,
+                int n_chunk_tiles, int n_tiles, int stages) {
+  using L = RouteTcLayout<NT>;
+  static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "UMMA N");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int KS = W / 64;
+  uint8_t *Qs = smem;
+  uint8_t *Ks = Qs + L::q_bytes(W);
+  float *Sb = reinterpret_cast<float *>(Ks + static_cast<size_t>(stages) * L::kSlice);
+  int *docs = reinterpret_cast<int *>(Sb + L::kTileC * L::kLD);
+  int *segs = docs + L::kTileC;  // kTileC + 1 run starts (+ padding)
+  uint64_t *bars = reinterpret_cast<uint64_t *>(segs + L::kTileC + 8);
+  // bars: full[stages], empty[stages], qfull, qempty, accf[2], acce[2], drain
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * stages + 7);
+  volatile int *fail = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + stages);
+  const uint32_t qfull = smem_u32(bars + 2 * stages), qempty = smem_u32(bars + 2 * stages + 1);
+  const uint32_t accf0 = smem_u32(bars + 2 * stages + 2), acce0 = smem_u32(bars + 2 * stages + 4);
+  const uint32_t drain = smem_u32(bars + 2 * stages + 6);
+  const uint32_t qs_addr = smem_u32(Qs), ks_addr = smem_u32(Ks);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(qfull, 1);
+    mbar_init(qempty, 1);
+    mbar_init(accf0, 1);
+    mbar_init(accf0 + 8, 1);
+    mbar_init(acce0, 128);
+    mbar_init(acce0 + 8, 128);
+    mbar_init(drain, 1);
+    *fail = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+  tc05_fence_before();
+  __syncthreads();
+  tc05_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    if (*fail) return false;
+    if (mbar_wait(bar, parity)) return true;
+    *fail = 1;
+    raise_device_error(MSA_DEVERR_WAIT_TIMEOUT);
+    return false;
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmQ);
+      const uint64_t pol = policy_evict_first();
+      int it = 0, qloads = 0, cur_rt = -1;
+      for (int tile = blockIdx.x; tile < n_tiles && !*fail; tile += gridDim.x) {
+        const int rt = tile / n_chunk_tiles, ct = tile % n_chunk_tiles;
+        if (rt != cur_rt) {
+          if (qloads > 0 && !wait(qempty, (qloads - 1) & 1)) break;
+          mbar_arrive_expect_tx(qfull, static_cast<uint32_t>(KS * NT * 128));
+          for (int s = 0; s < KS; ++s)
+            tma_load_2d(qs_addr + s * NT * 128, &tmQ, 64 * s, rt * NT, qfull);
+          ++qloads;
+          cur_rt = rt;
+        }
+        for (int s = 0; s < KS; ++s) {
+          const int st = it % stages;
+          if (it >= stages && !wait(empty0 + 8 * st, ((it / stages) - 1) & 1)) break;
+          mbar_arrive_expect_tx(full0 + 8 * st, L::kSlice);
+          tma_load_2d_hint(ks_addr + st * L::kSlice, &tmK, 64 * s, ct * L::kTileC,
+                           full0 + 8 * st, pol);
+          ++it;
+        }
+      }
+      if (*fail) {  // let every copy issued here land before the CTA can exit
+        for (int j = (it > stages ? it - stages : 0); j < it; ++j)
+          mbar_wait(full0 + 8 * (j % stages), (j / stages) & 1);
+        if (qloads > 0) mbar_wait(qfull, (qloads - 1) & 1);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16_f32<128, NT>();
+      int it = 0, quses = 0, cur_rt = -1, tl = 0;
+      bool issued = false;
+      for (int tile = blockIdx.x; tile < n_tiles && !*fail; tile += gridDim.x, ++tl) {
+        const int rt = tile / n_chunk_tiles;
+        if (rt != cur_rt) {
+          if (quses > 0) umma_commit(qempty);  // previous row tile's MMAs are all issued
+          if (!wait(qfull, quses & 1)) break;
+          ++quses;
+          cur_rt = rt;
+        }
+        const int buf = tl & 1;
+        if (tl >= 2 && !wait(acce0 + 8 * buf, ((tl >> 1) - 1) & 1)) break;
+        tc05_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * NT);
+        bool ok = true;
+        for (int s = 0; s < KS; ++s, ++it) {
+          const int st = it % stages;
+          if (!wait(full0 + 8 * st, (it / stages) & 1)) { ok = false; break; }
+          tc05_fence_after();
+          const uint32_t a0 = ks_addr + st * L::kSlice;
+          const uint32_t b0 = qs_addr + s * NT * 128;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(d_tmem, umma_desc_k_sw128(a0 + kk * 32), umma_desc_k_sw128(b0 + kk * 32),
+                      idesc, (s | kk) != 0);
+          umma_commit(empty0 + 8 * st);
+          issued = true;
+        }
+        if (!ok) break;
+        umma_commit(accf0 + 8 * buf);
+      }
+      if (issued) {  // every MMA has completed before TMEM can be freed
+        umma_commit(drain);
+        mbar_wait(drain, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int tid = threadIdx.x;  // 0..127 == TMEM lane == chunk row of the tile
+    int tl = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tl) {
+      const int rt = tile / n_chunk_tiles, ct = tile % n_chunk_tiles;
+      const int buf = tl & 1;
+      const int64_t c0 = static_cast<int64_t>(ct) * L::kTileC;
+      const int64_t r0 = static_cast<int64_t>(rt) * NT;
+      const int MC = static_cast<int>(C - c0 < L::kTileC ? C - c0 : L::kTileC);
+      const int NR = static_cast<int>(R - r0 < NT ? R - r0 : NT);
+      // the tile's document ids, loaded while the MMAs run
+      const int my_doc = tid < MC ? chunk_doc[c0 + tid] : 0;
+      const int prev_doc = c0 > 0 ? chunk_doc[c0 - 1] : -1;
+      const int next_doc = c0 + MC < C ? chunk_doc[c0 + MC] : -1;
+      const bool ok = wait(accf0 + 8 * buf, (tl >> 1) & 1);
+      tc05_fence_after();
+      if (ok) {
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) +
+                               static_cast<uint32_t>(buf * NT);
+#pragma unroll
+        for (int c = 0; c < NT; c += 16) {
+          float v[16];
+          tmem_ld16(taddr + c, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) Sb[tid * L::kLD + c + i] = v[i] * inv_Hr;
+        }
+      }
+      tc05_fence_before();
+      mbar_arrive(acce0 + 8 * buf);  // this accumulator may be overwritten
+      if (tid < MC) docs[tid] = my_doc;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // after a failed wait the results are void (the error word is set): skip the epilogue
+      const bool go = !*fail;
+      if (go) epi_token_max(Sb, L::kLD, MC, NR, r0, T_tok, tid, 128);
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int64_t b0 = r0 / T_tok;
+      const int QB = static_cast<int>((r0 + NR - 1) / T_tok - b0 + 1);
+      int q_lo, q_hi;
+      query_span(r0, NR, T_tok, b0, q_lo, q_hi);
+      epi_doc_max(Sb, L::kLD, MC, QB, b0, docs, prev_doc, next_doc, q_lo, q_hi, n_docs, state,
+                  segs, tid, 128, go);
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
+  }
+  tc05_fence_before();
+  __syncthreads();
+  tc05_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, L::kTmemCols);
+}
+
+}  // namespace msa

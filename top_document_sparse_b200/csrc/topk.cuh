@@ -11,6 +11,7 @@
 namespace msa {
 
 constexpr int kTopkThreads = 256;
+constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkPerThread = 16;
 constexpr int kTopkSlice = kTopkThreads * kTopkPerThread;  // documents per CTA
 
@@ -18,34 +19,27 @@ __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsig
   return a > b ? a : b;
 }
 
-// Block-wide max of one key per thread (kTopkThreads threads).
-__device__ __forceinline__ unsigned long long block_max_key(unsigned long long v,
-                                                            unsigned long long *red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = umax64(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    v = lane < kTopkThreads / 32 ? red[lane] : 0ull;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = umax64(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if (lane == 0) red[kTopkThreads / 32] = v;
-  }
-  __syncthreads();
-  return red[kTopkThreads / 32];
+// Warp-wide max of one 64-bit key per lane: max of the high words, then max of
+// the low words among the lanes holding that high word (two redux.sync).
+__device__ __forceinline__ unsigned long long warp_max_key(unsigned long long v) {
+  const unsigned hi = static_cast<unsigned>(v >> 32), lo = static_cast<unsigned>(v);
+  const unsigned hmax = __reduce_max_sync(0xffffffffu, hi);
+  const unsigned lmax = __reduce_max_sync(0xffffffffu, hi == hmax ? lo : 0u);
+  return (static_cast<unsigned long long>(hmax) << 32) | lmax;
 }
 
-// k rounds of "take the block's largest key"; only the owner rescans.
-// Key 0 means "no document" (never a valid key).
-__device__ __forceinline__ void select_topk(unsigned long long (&key)[kTopkPerThread], int k,
-                                            unsigned long long *out, unsigned long long *red) {
+// k rounds of "take the warp's largest key" over the lanes' key[] registers;
+// only the owner lane rescans.  Key 0 means "no document" (never a valid key).
+// Lane 0 writes the selection, largest first, to out[0..k).
+__device__ __forceinline__ void warp_select_topk(unsigned long long (&key)[kTopkPerThread], int k,
+                                                 unsigned long long *out) {
+  const int lane = threadIdx.x & 31;
   unsigned long long m = 0ull;
 #pragma unroll
   for (int j = 0; j < kTopkPerThread; ++j) m = umax64(m, key[j]);
   for (int r = 0; r < k; ++r) {
-    const unsigned long long w = block_max_key(m, red);
-    if (threadIdx.x == 0) out[r] = w;
+    const unsigned long long w = warp_max_key(m);
+    if (lane == 0) out[r] = w;
     if (w != 0ull && m == w) {
       m = 0ull;
 #pragma unroll
@@ -54,6 +48,25 @@ __device__ __forceinline__ void select_topk(unsigned long long (&key)[kTopkPerTh
         m = umax64(m, key[j]);
       }
     }
+  }
+}
+
+// Block top-k of the threads' key[] registers: every warp selects its own k,
+// then warp 0 selects k among the kTopkWarps * k candidates.  The result is
+// left in sel[0..k) (shared).
+__device__ __forceinline__ void block_select_topk(unsigned long long (&key)[kTopkPerThread], int k,
+                                                  unsigned long long *cand,
+                                                  unsigned long long *sel) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  warp_select_topk(key, k, cand + warp * k);
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int j = 0; j < kTopkPerThread; ++j) {
+      const int i = j * 32 + lane;
+      key[j] = i < kTopkWarps * k ? cand[i] : 0ull;
+    }
+    warp_select_topk(key, k, sel);
   }
   __syncthreads();
 }
@@ -67,24 +80,26 @@ __device__ __forceinline__ void write_topk(const unsigned long long *sel, int k,
   }
 }
 
-// grid (n_split, B).  With n_split == 1 the result goes straight to ids/scores.
+// grid (n_split, B).  Warp w of split s holds documents s*kTopkSlice + w*512 +
+// j*32 + lane.  With n_split == 1 the result goes straight to ids/scores.
 __global__ void __launch_bounds__(kTopkThreads)
 topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__ exclude,
                     int n_docs, int k, int n_split, unsigned long long *__restrict__ cand,
                     int32_t *__restrict__ ids, float *__restrict__ scores) {
-  __shared__ unsigned long long red[kTopkThreads / 32 + 1];
+  __shared__ unsigned long long wc[kTopkWarps * kMaxTopK];
   __shared__ unsigned long long sel[kMaxTopK];
   const int b = blockIdx.y, split = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(b) * n_docs;
   unsigned long long key[kTopkPerThread];
 #pragma unroll
   for (int j = 0; j < kTopkPerThread; ++j) {
-    const int d = split * kTopkSlice + j * kTopkThreads + threadIdx.x;
+    const int d = split * kTopkSlice + warp * (32 * kTopkPerThread) + j * 32 + lane;
     bool ok = d < n_docs;
     if (ok && exclude != nullptr) ok = exclude[row + d] == 0;
     key[j] = ok ? topk_key(state[row + d], d) : 0ull;
   }
-  select_topk(key, k, sel, red);
+  block_select_topk(key, k, wc, sel);
   if (n_split == 1) {
     write_topk(sel, k, ids + static_cast<int64_t>(b) * k, scores + static_cast<int64_t>(b) * k);
   } else {
@@ -97,16 +112,17 @@ topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__
 __global__ void __launch_bounds__(kTopkThreads)
 topk_merge_kernel(const unsigned long long *__restrict__ cand, int n_cand, int k,
                   int32_t *__restrict__ ids, float *__restrict__ scores) {
-  __shared__ unsigned long long red[kTopkThreads / 32 + 1];
+  __shared__ unsigned long long wc[kTopkWarps * kMaxTopK];
   __shared__ unsigned long long sel[kMaxTopK];
   const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned long long key[kTopkPerThread];
 #pragma unroll
   for (int j = 0; j < kTopkPerThread; ++j) {
-    const int i = j * kTopkThreads + threadIdx.x;
+    const int i = warp * (32 * kTopkPerThread) + j * 32 + lane;
     key[j] = i < n_cand ? cand[static_cast<int64_t>(b) * n_cand + i] : 0ull;
   }
-  select_topk(key, k, sel, red);
+  block_select_topk(key, k, wc, sel);
   write_topk(sel, k, ids + static_cast<int64_t>(b) * k, scores + static_cast<int64_t>(b) * k);
 }
 
