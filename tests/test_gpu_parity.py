@@ -2,7 +2,8 @@
 
 Tolerances (floating point): pooled means within 1e-6 x (mean |x| over the chunk) in fp32, plus
 one bf16 ulp when stored in bf16; routing scores 1e-5 (fp32) / 2e-3 (bf16) absolute; attention
-outputs 1e-5 (fp32) / 1e-2 (bf16) max-abs.  Top-k ids are compared exactly (as sets when the
+outputs 1e-5 (fp32) / 1e-2 (bf16) max-abs, the bf16 bound taken before the output's own rounding
+to bf16 (so + half a bf16 ulp of the expected value).  Top-k ids are compared exactly (as sets when the
 oracle's k-th / (k+1)-th gap is wider than twice the score tolerance, else checked for validity).
 """
 import numpy as np
@@ -20,6 +21,14 @@ pytestmark = pytest.mark.gpu
 
 SCORE_TOL = {"f32": 1e-5, "bf16": 2e-3}
 ATTN_TOL = {"f32": 1e-5, "bf16": 1e-2}
+
+
+def attn_tol(dt, want):
+    """The attention bound applies before the output is stored: a bf16 output adds up to half a
+    bf16 ulp of its own rounding (0.0078 at |O| ~ 2.6, where short local contexts put it)."""
+    if dt == "f32":
+        return ATTN_TOL["f32"]
+    return ATTN_TOL["bf16"] + 0.5 * bf16_ulp(to64(want))
 
 
 def _msa():
@@ -219,6 +228,11 @@ ATTN_CASES = [
     ("bf16", 64, 16, 16, 7, 1, 3),
     ("bf16", 128, 16, 1, 9, 2, 5),
     ("bf16", 64, 8, 4, 33, 1, 0),
+    # one-token decode kernel (head_dim 128, GQA group 2..16), with and without memory rows
+    ("bf16", 128, 16, 8, 20, 1, 3),
+    ("bf16", 128, 64, 8, 11, 1, 2),
+    ("bf16", 128, 32, 2, 5, 1, 4),
+    ("bf16", 128, 32, 8, 40, 1, 0),
 ]
 
 
@@ -255,7 +269,7 @@ def test_attend_matches_oracle(dt, D, H_q, H_kv, T0, T1, k):
         ref, _, rs = oracle.attend(Q[:, sl], Kn[:, :start + T], Vn[:, :start + T], start, Kb, Vb,
                                    mem.doc_chunk_offsets, ids_np, pos_offset, w.rope_theta)
         np.testing.assert_allclose(rs, 1.0, atol=1e-12)
-        assert_close(O, ref, tol, f"attention output (tokens {start}..{start + T})")
+        assert_close(O, ref, attn_tol(dt, ref), f"attention output (tokens {start}..{start + T})")
         start += T
         assert clen.cpu().tolist() == [start] * B
     assert msa.device_error() == 0
@@ -301,7 +315,7 @@ def test_decode_steps_match_oracle():
         _check_topk(layer.ids, layer.scores, layer.state, st, k, SCORE_TOL["bf16"])
         # same set; the rank order among near-equal scores changes only rounding
         assert set(layer.ids.cpu().numpy()[0].tolist()) == set(ids_o[0].tolist())
-        assert_close(Ot, O_ref, ATTN_TOL["bf16"], f"decode output, step {s}")
+        assert_close(Ot, O_ref, attn_tol("bf16", O_ref), f"decode output, step {s}")
     assert layer.cache_len.cpu().tolist() == [T + n_steps]
     assert msa.device_error() == 0
 

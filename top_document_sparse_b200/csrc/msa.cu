@@ -214,6 +214,20 @@ msa_status launch_route_tc(const msa_memory *mem, const void *keys, const void *
   return MSA_OK;
 }
 
+template <int KL>
+msa_status launch_topk(const msa_memory *mem, const float *state, const uint8_t *exclude, int B,
+                       int k, int n_split, unsigned long long *cand, int32_t *ids, float *scores,
+                       cudaStream_t st) {
+  msa::topk_partial_kernel<KL><<<dim3(n_split, B), msa::kTopkThreads, 0, st>>>(
+      state, exclude, mem->n_docs, k, n_split, cand, ids, scores);
+  MSA_LAUNCHED("topk_partial_kernel");
+  if (n_split > 1) {
+    msa::topk_merge_kernel<KL><<<B, msa::kTopkThreads, 0, st>>>(cand, n_split * k, k, ids, scores);
+    MSA_LAUNCHED("topk_merge_kernel");
+  }
+  return MSA_OK;
+}
+
 msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, int B, int T, int k,
                       const uint8_t *exclude, float *state, int32_t *ids, float *scores,
                       void *ws, size_t ws_bytes, cudaStream_t st) {
@@ -266,14 +280,9 @@ msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, i
   }
   auto *cand = reinterpret_cast<unsigned long long *>(wsb + plan.cand);
   if (B > 65535) return fail(MSA_ERR_UNSUPPORTED, "batch too large for top-k");
-  msa::topk_partial_kernel<<<dim3(plan.n_split, B), msa::kTopkThreads, 0, st>>>(
-      state, exclude, mem->n_docs, k, plan.n_split, cand, ids, scores);
-  MSA_LAUNCHED("topk_partial_kernel");
-  if (plan.n_split > 1) {
-    msa::topk_merge_kernel<<<B, msa::kTopkThreads, 0, st>>>(cand, plan.n_split * k, k, ids, scores);
-    MSA_LAUNCHED("topk_merge_kernel");
-  }
-  return MSA_OK;
+  if (k <= 16) return launch_topk<16>(mem, state, exclude, B, k, plan.n_split, cand, ids, scores, st);
+  if (k <= 32) return launch_topk<32>(mem, state, exclude, B, k, plan.n_split, cand, ids, scores, st);
+  return launch_topk<64>(mem, state, exclude, B, k, plan.n_split, cand, ids, scores, st);
 }
 
 template <int D, int G>

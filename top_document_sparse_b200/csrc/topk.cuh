@@ -19,54 +19,87 @@ __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsig
   return a > b ? a : b;
 }
 
-// Warp-wide max of one 64-bit key per lane: max of the high words, then max of
-// the low words among the lanes holding that high word (two redux.sync).
-__device__ __forceinline__ unsigned long long warp_max_key(unsigned long long v) {
-  const unsigned hi = static_cast<unsigned>(v >> 32), lo = static_cast<unsigned>(v);
-  const unsigned hmax = __reduce_max_sync(0xffffffffu, hi);
-  const unsigned lmax = __reduce_max_sync(0xffffffffu, hi == hmax ? lo : 0u);
-  return (static_cast<unsigned long long>(hmax) << 32) | lmax;
+// --- sorting-network selection ------------------------------------------
+// Each lane keeps a list of KL keys sorted in descending order.  Two lanes'
+// lists are combined into the KL largest of their union by reversing one list,
+// taking elementwise maxima (a bitonic sequence holding the KL largest) and
+// sorting that with a bitonic merge network.  Five such butterfly rounds over
+// the warp leave every lane with the warp's KL largest keys; no step depends
+// on k serially.
+
+template <int KL>
+__device__ __forceinline__ void cas_desc(unsigned long long (&a)[KL], int i, int j) {
+  const unsigned long long x = a[i], y = a[j];
+  a[i] = x > y ? x : y;
+  a[j] = x > y ? y : x;
 }
 
-// k rounds of "take the warp's largest key" over the lanes' key[] registers;
-// only the owner lane rescans.  Key 0 means "no document" (never a valid key).
-// Lane 0 writes the selection, largest first, to out[0..k).
-__device__ __forceinline__ void warp_select_topk(unsigned long long (&key)[kTopkPerThread], int k,
-                                                 unsigned long long *out) {
-  const int lane = threadIdx.x & 31;
-  unsigned long long m = 0ull;
+// full bitonic sort, descending, of a[0..KL)
+template <int KL>
+__device__ __forceinline__ void sort_desc(unsigned long long (&a)[KL]) {
 #pragma unroll
-  for (int j = 0; j < kTopkPerThread; ++j) m = umax64(m, key[j]);
-  for (int r = 0; r < k; ++r) {
-    const unsigned long long w = warp_max_key(m);
-    if (lane == 0) out[r] = w;
-    if (w != 0ull && m == w) {
-      m = 0ull;
+  for (int size = 2; size <= KL; size <<= 1)
 #pragma unroll
-      for (int j = 0; j < kTopkPerThread; ++j) {
-        if (key[j] == w) key[j] = 0ull;
-        m = umax64(m, key[j]);
+    for (int stride = size >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+      for (int i = 0; i < KL; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          // descending within blocks whose (i & size) == 0, ascending otherwise
+          if ((i & size) == 0) cas_desc<KL>(a, i, j); else cas_desc<KL>(a, j, i);
+        }
       }
-    }
-  }
 }
 
-// Block top-k of the threads' key[] registers: every warp selects its own k,
-// then warp 0 selects k among the kTopkWarps * k candidates.  The result is
-// left in sel[0..k) (shared).
-__device__ __forceinline__ void block_select_topk(unsigned long long (&key)[kTopkPerThread], int k,
-                                                  unsigned long long *cand,
+// a bitonic sequence -> sorted descending
+template <int KL>
+__device__ __forceinline__ void bitonic_merge_desc(unsigned long long (&a)[KL]) {
+#pragma unroll
+  for (int stride = KL >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+    for (int i = 0; i < KL; ++i) {
+      const int j = i ^ stride;
+      if (j > i) cas_desc<KL>(a, i, j);
+    }
+}
+
+// the KL largest of this lane's list and the list of lane ^ offset
+template <int KL>
+__device__ __forceinline__ void merge_with_lane(unsigned long long (&a)[KL], int offset) {
+  unsigned long long b[KL];
+#pragma unroll
+  for (int i = 0; i < KL; ++i) b[i] = __shfl_xor_sync(0xffffffffu, a[KL - 1 - i], offset);
+#pragma unroll
+  for (int i = 0; i < KL; ++i) a[i] = a[i] > b[i] ? a[i] : b[i];
+  bitonic_merge_desc<KL>(a);
+}
+
+// Block top-k (k <= KL) of the threads' key[] registers (kTopkPerThread each):
+// per-lane sort, warp butterflies, then warp 0 merges the warps' lists.  The
+// k largest keys, descending, end in sel[0..k).
+template <int KL>
+__device__ __forceinline__ void block_select_topk(const unsigned long long (&key)[kTopkPerThread],
+                                                  int k, unsigned long long *cand,
                                                   unsigned long long *sel) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  warp_select_topk(key, k, cand + warp * k);
+  unsigned long long a[KL];
+#pragma unroll
+  for (int i = 0; i < KL; ++i) a[i] = i < kTopkPerThread ? key[i] : 0ull;
+  sort_desc<KL>(a);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) merge_with_lane<KL>(a, o);
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < KL; ++i) cand[warp * KL + i] = a[i];
+  }
   __syncthreads();
   if (warp == 0) {
 #pragma unroll
-    for (int j = 0; j < kTopkPerThread; ++j) {
-      const int i = j * 32 + lane;
-      key[j] = i < kTopkWarps * k ? cand[i] : 0ull;
-    }
-    warp_select_topk(key, k, sel);
+    for (int i = 0; i < KL; ++i) a[i] = lane < kTopkWarps ? cand[lane * KL + i] : 0ull;
+#pragma unroll
+    for (int o = kTopkWarps >> 1; o > 0; o >>= 1) merge_with_lane<KL>(a, o);
+    if (lane == 0)
+      for (int i = 0; i < k; ++i) sel[i] = a[i];
   }
   __syncthreads();
 }
@@ -82,11 +115,12 @@ __device__ __forceinline__ void write_topk(const unsigned long long *sel, int k,
 
 // grid (n_split, B).  Warp w of split s holds documents s*kTopkSlice + w*512 +
 // j*32 + lane.  With n_split == 1 the result goes straight to ids/scores.
+template <int KL>
 __global__ void __launch_bounds__(kTopkThreads)
 topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__ exclude,
                     int n_docs, int k, int n_split, unsigned long long *__restrict__ cand,
                     int32_t *__restrict__ ids, float *__restrict__ scores) {
-  __shared__ unsigned long long wc[kTopkWarps * kMaxTopK];
+  __shared__ unsigned long long wc[kTopkWarps * KL];
   __shared__ unsigned long long sel[kMaxTopK];
   const int b = blockIdx.y, split = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -99,7 +133,7 @@ topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__
     if (ok && exclude != nullptr) ok = exclude[row + d] == 0;
     key[j] = ok ? topk_key(state[row + d], d) : 0ull;
   }
-  block_select_topk(key, k, wc, sel);
+  block_select_topk<KL>(key, k, wc, sel);
   if (n_split == 1) {
     write_topk(sel, k, ids + static_cast<int64_t>(b) * k, scores + static_cast<int64_t>(b) * k);
   } else {
@@ -109,10 +143,11 @@ topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__
 }
 
 // grid (B).  n_cand = n_split * k <= kTopkSlice.
+template <int KL>
 __global__ void __launch_bounds__(kTopkThreads)
 topk_merge_kernel(const unsigned long long *__restrict__ cand, int n_cand, int k,
                   int32_t *__restrict__ ids, float *__restrict__ scores) {
-  __shared__ unsigned long long wc[kTopkWarps * kMaxTopK];
+  __shared__ unsigned long long wc[kTopkWarps * KL];
   __shared__ unsigned long long sel[kMaxTopK];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -122,7 +157,7 @@ topk_merge_kernel(const unsigned long long *__restrict__ cand, int n_cand, int k
     const int i = warp * (32 * kTopkPerThread) + j * 32 + lane;
     key[j] = i < n_cand ? cand[static_cast<int64_t>(b) * n_cand + i] : 0ull;
   }
-  block_select_topk(key, k, wc, sel);
+  block_select_topk<KL>(key, k, wc, sel);
   write_topk(sel, k, ids + static_cast<int64_t>(b) * k, scores + static_cast<int64_t>(b) * k);
 }
 
