@@ -285,6 +285,65 @@ MSA_API msa_status msa_step(const msa_memory *mem, const void *router_keys,
                     const void *Qr_tok, const void *Q_tok, const void *K_tok,
                     const void *V_tok, void *O_tok, msa_stream stream);
 
+/*
+ * Host tier of the pooled content [Evermind summary sec. 4B "Memory Parallel &
+ * Tiered Storage": routing keys stay in GPU memory, the content K/V stays in
+ * host DRAM and only the selected documents are fetched, asynchronously;
+ * b-lab.team item 2, KV cache compression].
+ *
+ * A fetcher manages a device slot cache for one layer's content:
+ *   content_host : PINNED host memory [C][2][H_kv][D] written by
+ *                  msa_encode_memory (it may write host memory directly)
+ *   slot_cache   : device memory of n_slots * doc_content_stride bytes
+ *                  (msa_memory_get_info), one document per slot
+ *   n_slots      : >= max_batch * max_k, so one call's documents always fit
+ *   flags        : MSA_FETCH_COLD forgets every resident document at each
+ *                  fetch (every selected document crosses the host link)
+ * The fetcher allocates small host-side tables, two events, pinned host
+ * staging for max_batch * max_k ids and slots, and a device array of the same
+ * size; it does not own content_host or slot_cache.
+ */
+typedef struct msa_fetcher msa_fetcher;
+#define MSA_FETCH_COLD 0x1u
+
+MSA_API msa_status msa_fetcher_create(const msa_memory *mem, const void *content_host,
+                                      void *slot_cache, int32_t n_slots, int32_t max_batch,
+                                      int32_t max_k, uint32_t flags, msa_fetcher **out);
+MSA_API msa_status msa_fetcher_destroy(msa_fetcher *f);
+/* Totals since creation: (query, rank) hits and misses, documents copied,
+ * bytes copied over the host link. */
+MSA_API msa_status msa_fetcher_stats(const msa_fetcher *f, int64_t *hits, int64_t *misses,
+                                     int64_t *copies, int64_t *bytes);
+
+/*
+ * Make the documents ids[batch][k] (device) resident in the slot cache.
+ * Reads the ids back to the host (synchronising `stream` up to that copy),
+ * keeps resident documents, chooses victim slots (a clock over the slots not
+ * used by this call) for the others and copies each missing document (one
+ * cudaMemcpyAsync of its contiguous chunk rows) on `fetch_stream`, uploads
+ * the slot of every (query, rank), and makes `stream` wait for
+ * `fetch_stream`.  Ids outside [0, n_docs) get slot 0 and are skipped by the
+ * attention (device error word).  fetch_stream may equal stream.
+ */
+MSA_API msa_status msa_fetch(msa_fetcher *f, const int32_t *ids, int32_t batch, int32_t k,
+                             msa_stream stream, msa_stream fetch_stream);
+
+/* msa_sparse_attend over the memory rows the last msa_fetch of `f` placed in
+ * its slot cache (same ids, batch and k). */
+MSA_API msa_status msa_sparse_attend_fetched(
+    const msa_memory *mem, const msa_fetcher *f, const int32_t *ids, int32_t batch, int32_t k,
+    int32_t tokens, int32_t n_q_heads, const void *Q, const void *K_new, const void *V_new,
+    void *K_cache, void *V_cache, int32_t *cache_len, int32_t cache_capacity,
+    int32_t pos_offset, void *O, void *workspace, size_t workspace_bytes, msa_stream stream);
+
+/* msa_step with the content in the host tier: route, msa_fetch, then the
+ * attention over the fetched rows.  Synchronises `stream` once (the id
+ * read-back). */
+MSA_API msa_status msa_step_host(const msa_memory *mem, const void *router_keys, msa_fetcher *f,
+                                 const msa_decode_state *st, const void *Qr_tok,
+                                 const void *Q_tok, const void *K_tok, const void *V_tok,
+                                 void *O_tok, msa_stream stream, msa_stream fetch_stream);
+
 /* Read and clear the device error word of the current device (synchronises
  * `stream`).  *bits receives the MSA_DEVERR_* bits; returns MSA_ERR_TIMEOUT or
  * MSA_ERR_STATE when a bit was set, else MSA_OK. */

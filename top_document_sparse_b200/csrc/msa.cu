@@ -14,6 +14,7 @@
 #include "pool.cuh"
 #include "route.cuh"
 #include "route_tc.cuh"
+#include "tier.cuh"
 #include "topk.cuh"
 
 // Scratch of msa_sparse_attend_static: a fixed device array, so that callers
@@ -694,6 +695,177 @@ msa_status msa_step(const msa_memory *mem, const void *router_keys, const void *
   return attend_impl(mem, content, s->ids, nullptr, 0, s->batch, s->top_k, 1, s->n_q_heads, Q_tok,
                      K_tok, V_tok, s->k_cache, s->v_cache, s->cache_len, s->cache_capacity,
                      s->pos_offset, O_tok, ws + route_bytes, s->workspace_bytes - route_bytes, st);
+}
+
+msa_status msa_fetcher_create(const msa_memory *mem, const void *content_host, void *slot_cache,
+                              int32_t n_slots, int32_t max_batch, int32_t max_k, uint32_t flags,
+                              msa_fetcher **out) {
+  if (!mem || !content_host || !slot_cache || !out)
+    return fail(MSA_ERR_INVALID_ARG, "null argument");
+  *out = nullptr;
+  if (max_batch < 1 || max_k < 1 || max_k > msa::kMaxTopK)
+    return fail(MSA_ERR_INVALID_ARG, "max_batch >= 1 and 1 <= max_k <= %d required", msa::kMaxTopK);
+  if (static_cast<int64_t>(n_slots) < static_cast<int64_t>(max_batch) * max_k)
+    return fail(MSA_ERR_INVALID_ARG, "n_slots=%d < max_batch * max_k = %lld", n_slots,
+                (long long)max_batch * max_k);
+  if (!aligned16(slot_cache)) return fail(MSA_ERR_INVALID_ARG, "slot cache must be 16-byte aligned");
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, content_host) != cudaSuccess ||
+      attr.type != cudaMemoryTypeHost) {
+    cudaGetLastError();
+    return fail(MSA_ERR_INVALID_ARG, "content_host must be pinned (page-locked) host memory");
+  }
+  auto f = new msa_fetcher();
+  f->mem = mem;
+  f->content_host = static_cast<const uint8_t *>(content_host);
+  f->slot_cache = static_cast<uint8_t *>(slot_cache);
+  f->n_slots = n_slots;
+  f->max_batch = max_batch;
+  f->max_k = max_k;
+  f->flags = flags;
+  f->row_bytes = static_cast<size_t>(2) * mem->H_kv * mem->D * elem_size(mem->dtype);
+  f->slot_bytes = f->row_bytes * mem->max_doc_chunks;
+  f->doc_slot.assign(mem->n_docs, -1);
+  f->slot_doc.assign(n_slots, -1);
+  f->slot_stamp.assign(n_slots, 0);
+  const size_t n = static_cast<size_t>(max_batch) * max_k;
+  if (cudaHostAlloc(reinterpret_cast<void **>(&f->h_ids), n * 4, cudaHostAllocDefault) != cudaSuccess ||
+      cudaHostAlloc(reinterpret_cast<void **>(&f->h_slots), n * 4, cudaHostAllocDefault) != cudaSuccess ||
+      cudaMalloc(reinterpret_cast<void **>(&f->d_slots), n * 4) != cudaSuccess ||
+      cudaEventCreateWithFlags(&f->ev_ids, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&f->ev_fetch, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    msa_fetcher_destroy(f);
+    return fail(MSA_ERR_OUT_OF_MEMORY, "could not allocate the fetcher's staging buffers");
+  }
+  *out = f;
+  return MSA_OK;
+}
+
+msa_status msa_fetcher_destroy(msa_fetcher *f) {
+  if (!f) return fail(MSA_ERR_INVALID_ARG, "null fetcher");
+  if (f->h_ids) cudaFreeHost(f->h_ids);
+  if (f->h_slots) cudaFreeHost(f->h_slots);
+  if (f->d_slots) cudaFree(f->d_slots);
+  if (f->ev_ids) cudaEventDestroy(f->ev_ids);
+  if (f->ev_fetch) cudaEventDestroy(f->ev_fetch);
+  delete f;
+  return MSA_OK;
+}
+
+msa_status msa_fetcher_stats(const msa_fetcher *f, int64_t *hits, int64_t *misses,
+                             int64_t *copies, int64_t *bytes) {
+  if (!f) return fail(MSA_ERR_INVALID_ARG, "null fetcher");
+  if (hits) *hits = f->hits;
+  if (misses) *misses = f->misses;
+  if (copies) *copies = f->copies;
+  if (bytes) *bytes = f->bytes;
+  return MSA_OK;
+}
+
+msa_status msa_fetch(msa_fetcher *f, const int32_t *ids, int32_t batch, int32_t k,
+                     msa_stream stream, msa_stream fetch_stream) {
+  if (!f || !ids) return fail(MSA_ERR_INVALID_ARG, "null fetcher or ids");
+  if (batch < 1 || batch > f->max_batch || k < 1 || k > f->max_k)
+    return fail(MSA_ERR_INVALID_ARG, "batch=%d k=%d beyond the fetcher's %d x %d", batch, k,
+                f->max_batch, f->max_k);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t fst = reinterpret_cast<cudaStream_t>(fetch_stream);
+  const int n = batch * k;
+  MSA_CUDA(cudaMemcpyAsync(f->h_ids, ids, n * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  MSA_CUDA(cudaEventRecord(f->ev_ids, st));
+  MSA_CUDA(cudaEventSynchronize(f->ev_ids));
+  const int64_t now = ++f->stamp;
+  if (f->flags & MSA_FETCH_COLD) {
+    for (int s = 0; s < f->n_slots; ++s) {
+      if (f->slot_doc[s] >= 0) f->doc_slot[f->slot_doc[s]] = -1;
+      f->slot_doc[s] = -1;
+    }
+  }
+  const msa_memory *mem = f->mem;
+  // resident documents keep their slots
+  for (int i = 0; i < n; ++i) {
+    const int d = f->h_ids[i];
+    if (d < 0 || d >= mem->n_docs) continue;
+    const int s = f->doc_slot[d];
+    if (s >= 0) f->slot_stamp[s] = now;
+  }
+  for (int i = 0; i < n; ++i) {
+    const int d = f->h_ids[i];
+    if (d < 0 || d >= mem->n_docs) {
+      f->h_slots[i] = 0;
+      continue;
+    }
+    int s = f->doc_slot[d];
+    if (s >= 0 && f->slot_stamp[s] == now) {
+      f->h_slots[i] = s;
+      ++f->hits;
+      continue;
+    }
+    // a clock over the slots this call has not claimed (n_slots >= n guarantees one)
+    while (f->slot_stamp[f->hand] == now) f->hand = (f->hand + 1) % f->n_slots;
+    s = f->hand;
+    f->hand = (f->hand + 1) % f->n_slots;
+    if (f->slot_doc[s] >= 0) f->doc_slot[f->slot_doc[s]] = -1;
+    f->slot_doc[s] = d;
+    f->doc_slot[d] = s;
+    f->slot_stamp[s] = now;
+    f->h_slots[i] = s;
+    const int64_t c0 = mem->doc_chunk_off[d], c1 = mem->doc_chunk_off[d + 1];
+    const size_t nb = static_cast<size_t>(c1 - c0) * f->row_bytes;
+    MSA_CUDA(cudaMemcpyAsync(f->slot_cache + static_cast<size_t>(s) * f->slot_bytes,
+                             f->content_host + static_cast<size_t>(c0) * f->row_bytes, nb,
+                             cudaMemcpyHostToDevice, fst));
+    ++f->misses;
+    ++f->copies;
+    f->bytes += static_cast<int64_t>(nb);
+  }
+  MSA_CUDA(cudaMemcpyAsync(f->d_slots, f->h_slots, n * sizeof(int32_t), cudaMemcpyHostToDevice, fst));
+  if (fst != st) {
+    MSA_CUDA(cudaEventRecord(f->ev_fetch, fst));
+    MSA_CUDA(cudaStreamWaitEvent(st, f->ev_fetch, 0));
+  }
+  return MSA_OK;
+}
+
+msa_status msa_sparse_attend_fetched(const msa_memory *mem, const msa_fetcher *f,
+                                     const int32_t *ids, int32_t batch, int32_t k, int32_t tokens,
+                                     int32_t n_q_heads, const void *Q, const void *K_new,
+                                     const void *V_new, void *K_cache, void *V_cache,
+                                     int32_t *cache_len, int32_t cache_capacity,
+                                     int32_t pos_offset, void *O, void *workspace,
+                                     size_t workspace_bytes, msa_stream stream) {
+  if (!mem || !f) return fail(MSA_ERR_INVALID_ARG, "null memory or fetcher");
+  if (f->mem != mem) return fail(MSA_ERR_INVALID_ARG, "fetcher belongs to another memory");
+  if (batch > f->max_batch || k > f->max_k)
+    return fail(MSA_ERR_INVALID_ARG, "batch / k beyond the fetcher's sizes");
+  return attend_impl(mem, f->slot_cache, ids, f->d_slots, mem->max_doc_chunks, batch, k, tokens,
+                     n_q_heads, Q, K_new, V_new, K_cache, V_cache, cache_len, cache_capacity,
+                     pos_offset, O, workspace, workspace_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+msa_status msa_step_host(const msa_memory *mem, const void *router_keys, msa_fetcher *f,
+                         const msa_decode_state *s, const void *Qr_tok, const void *Q_tok,
+                         const void *K_tok, const void *V_tok, void *O_tok, msa_stream stream,
+                         msa_stream fetch_stream) {
+  if (!mem || !s || !f) return fail(MSA_ERR_INVALID_ARG, "null memory, decode state or fetcher");
+  const size_t need = msa_step_workspace_size(mem, s->batch, s->top_k, s->n_q_heads);
+  if (s->workspace_bytes < need || !s->workspace)
+    return fail(MSA_ERR_INVALID_ARG, "decode workspace too small: %zu < %zu", s->workspace_bytes,
+                need);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t route_bytes = round256(plan_route(mem, s->batch, 1, s->top_k).bytes);
+  uint8_t *ws = static_cast<uint8_t *>(s->workspace);
+  msa_status r = route_impl(mem, router_keys, Qr_tok, s->batch, 1, s->top_k, nullptr, s->state,
+                            s->ids, s->scores, ws, route_bytes, st);
+  if (r != MSA_OK) return r;
+  r = msa_fetch(f, s->ids, s->batch, s->top_k, stream, fetch_stream);
+  if (r != MSA_OK) return r;
+  return attend_impl(mem, f->slot_cache, s->ids, f->d_slots, mem->max_doc_chunks, s->batch,
+                     s->top_k, 1, s->n_q_heads, Q_tok, K_tok, V_tok, s->k_cache, s->v_cache,
+                     s->cache_len, s->cache_capacity, s->pos_offset, O_tok, ws + route_bytes,
+                     s->workspace_bytes - route_bytes, st);
 }
 
 msa_status msa_device_error(uint32_t *bits, msa_stream stream) {

@@ -77,6 +77,16 @@ SIGNATURES = {
                                                 _P, _P, _P, _I32, _I32, _P, _P]),
     "msa_step_workspace_size": (_SZ, [_P, _I32, _I32, _I32]),
     "msa_step": (ctypes.c_int, [_P, _P, _P, ctypes.POINTER(DecodeState), _P, _P, _P, _P, _P, _P]),
+    "msa_fetcher_create": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, ctypes.c_uint32,
+                                          ctypes.POINTER(_P)]),
+    "msa_fetcher_destroy": (ctypes.c_int, [_P]),
+    "msa_fetcher_stats": (ctypes.c_int, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
+                                         ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),
+    "msa_fetch": (ctypes.c_int, [_P, _P, _I32, _I32, _P, _P]),
+    "msa_sparse_attend_fetched": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P,
+                                                 _P, _P, _P, _I32, _I32, _P, _P, _SZ, _P]),
+    "msa_step_host": (ctypes.c_int, [_P, _P, _P, ctypes.POINTER(DecodeState), _P, _P, _P, _P, _P,
+                                     _P, _P]),
     "msa_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "msa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "msa_last_error": (ctypes.c_char_p, []),
@@ -236,6 +246,68 @@ class Memory:
         _check(_lib.msa_step(self.handle, _ptr(router_keys), _ptr(content), ctypes.byref(st.c),
                              _ptr(Qr_tok), _ptr(Q_tok), _ptr(K_tok), _ptr(V_tok), _ptr(O_tok),
                              _stream(stream)))
+
+
+FETCH_COLD = 0x1
+
+
+class Fetcher:
+    """Host tier of one layer's pooled content: pinned host content plus a device slot cache
+    (msa_fetcher_*).  Owns neither buffer; keeps references so they outlive it."""
+
+    def __init__(self, mem: Memory, content_host: torch.Tensor, n_slots: int, max_batch: int,
+                 max_k: int, cold: bool = False, device="cuda"):
+        if not content_host.is_pinned():
+            raise ValueError("content_host must be pinned host memory")
+        self.mem = mem
+        self.content_host = content_host
+        self.slot_cache = torch.empty(n_slots * mem.info.doc_content_stride, dtype=torch.uint8,
+                                      device=device)
+        h = _P()
+        _check(_lib.msa_fetcher_create(mem.handle, content_host.data_ptr(),
+                                       self.slot_cache.data_ptr(), n_slots, max_batch, max_k,
+                                       FETCH_COLD if cold else 0, ctypes.byref(h)))
+        self.handle = h
+
+    def close(self):
+        if getattr(self, "handle", None):
+            _check(_lib.msa_fetcher_destroy(self.handle))
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def stats(self) -> dict:
+        v = [_I64() for _ in range(4)]
+        _check(_lib.msa_fetcher_stats(self.handle, *[ctypes.byref(x) for x in v]))
+        return dict(zip(("hits", "misses", "copies", "bytes"), (x.value for x in v)))
+
+    def fetch(self, ids, stream=None, fetch_stream=None):
+        B, k = ids.shape
+        _check(_lib.msa_fetch(self.handle, _ptr(ids), B, k, _stream(stream),
+                              _stream(fetch_stream) if fetch_stream is not None else _stream(stream)))
+
+    def sparse_attend(self, ids, Q, K_new, V_new, K_cache, V_cache, cache_len, pos_offset: int,
+                      O, workspace, stream=None):
+        B, T, H_q, _ = Q.shape
+        k = ids.shape[1]
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        _check(_lib.msa_sparse_attend_fetched(self.mem.handle, self.handle, _ptr(ids), B, k, T, H_q,
+                                              _ptr(Q), _ptr(K_new), _ptr(V_new), _ptr(K_cache),
+                                              _ptr(V_cache), _ptr(cache_len), K_cache.shape[1],
+                                              pos_offset, _ptr(O), _ptr(workspace), ws_bytes,
+                                              _stream(stream)))
+
+    def step(self, router_keys, st: "LayerDecode", Qr_tok, Q_tok, K_tok, V_tok, O_tok,
+             stream=None, fetch_stream=None):
+        _check(_lib.msa_step_host(self.mem.handle, _ptr(router_keys), self.handle,
+                                  ctypes.byref(st.c), _ptr(Qr_tok), _ptr(Q_tok), _ptr(K_tok),
+                                  _ptr(V_tok), _ptr(O_tok), _stream(stream),
+                                  _stream(fetch_stream) if fetch_stream is not None
+                                  else _stream(stream)))
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
