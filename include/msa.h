@@ -286,6 +286,30 @@ MSA_API msa_status msa_step(const msa_memory *mem, const void *router_keys,
                     const void *V_tok, void *O_tok, msa_stream stream);
 
 /*
+ * Memory Interleave [Evermind summary sec. 4C; b-lab.team item 3: generative
+ * retrieval -> context expansion -> generation, repeated; the documents
+ * retrieved in one round become part of the query of the next].  Runs
+ * `rounds` routing rounds for every query of the batch:
+ *   round 0 routes Qr [batch][tokens][H_r][d_r];
+ *   round r > 0 routes the unit router rows (every chunk, every head) of the
+ *   documents retrieved in round r-1;
+ * each with the running state carried over, and each round's top-k taken
+ * among the documents not yet in the context (taken[b][d] == 0).
+ *   state  : device [batch][n_docs] fp32, reset to -inf here
+ *   taken  : device [batch][n_docs] uint8, reset to 0 here; on return it marks
+ *            every document retrieved in rounds 0..rounds-2
+ *   ids, scores : device [rounds][batch][k]
+ * The next round's row count is read back to the host once per round.
+ */
+MSA_API size_t msa_interleave_workspace_size(const msa_memory *mem, int32_t batch,
+                                             int32_t tokens, int32_t k);
+MSA_API msa_status msa_interleave(const msa_memory *mem, const void *router_keys,
+                                  const void *Qr, int32_t batch, int32_t tokens, int32_t k,
+                                  int32_t rounds, float *state, uint8_t *taken, int32_t *ids,
+                                  float *scores, void *workspace, size_t workspace_bytes,
+                                  msa_stream stream);
+
+/*
  * Host tier of the pooled content [Evermind summary sec. 4B "Memory Parallel &
  * Tiered Storage": routing keys stay in GPU memory, the content K/V stays in
  * host DRAM and only the selected documents are fetched, asynchronously;

@@ -231,7 +231,8 @@ msa_status launch_topk(const msa_memory *mem, const float *state, const uint8_t 
 
 msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, int B, int T, int k,
                       const uint8_t *exclude, float *state, int32_t *ids, float *scores,
-                      void *ws, size_t ws_bytes, cudaStream_t st) {
+                      void *ws, size_t ws_bytes, cudaStream_t st, int q_pitch = 0) {
+  if (q_pitch <= 0) q_pitch = T;
   if (!mem) return fail(MSA_ERR_INVALID_ARG, "null memory");
   if (B < 1 || T < 0) return fail(MSA_ERR_INVALID_ARG, "batch must be >= 1 and tokens >= 0");
   if (k < 1 || k > mem->n_docs || k > msa::kMaxTopK)
@@ -257,7 +258,7 @@ msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, i
     if (mem->dtype == MSA_BF16) {
       auto *qh = reinterpret_cast<__nv_bfloat16 *>(wsb + plan.qhat);
       msa::qnorm_kernel<__nv_bfloat16><<<R, thr, 0, st>>>(
-          static_cast<const __nv_bfloat16 *>(Qr), W, mem->d_r, qh);
+          static_cast<const __nv_bfloat16 *>(Qr), W, mem->d_r, T, q_pitch, qh);
       MSA_LAUNCHED("qnorm_kernel");
       msa_status s;
       if (R <= 16)
@@ -269,7 +270,8 @@ msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, i
       if (s != MSA_OK) return s;
     } else {
       auto *qh = reinterpret_cast<float *>(wsb + plan.qhat);
-      msa::qnorm_kernel<float><<<R, thr, 0, st>>>(static_cast<const float *>(Qr), W, mem->d_r, qh);
+      msa::qnorm_kernel<float><<<R, thr, 0, st>>>(static_cast<const float *>(Qr), W, mem->d_r, T,
+                                                  q_pitch, qh);
       MSA_LAUNCHED("qnorm_kernel");
       dim3 grid(static_cast<unsigned>((mem->n_chunks + 31) / 32), static_cast<unsigned>((R + 31) / 32));
       if (grid.y > 65535) return fail(MSA_ERR_UNSUPPORTED, "too many query rows for fp32 route");
@@ -866,6 +868,92 @@ msa_status msa_step_host(const msa_memory *mem, const void *router_keys, msa_fet
                      s->top_k, 1, s->n_q_heads, Q_tok, K_tok, V_tok, s->k_cache, s->v_cache,
                      s->cache_len, s->cache_capacity, s->pos_offset, O_tok, ws + route_bytes,
                      s->workspace_bytes - route_bytes, st);
+}
+
+// Workspace of msa_interleave: the route workspace for the largest round, the
+// gathered rows [batch][k * max_doc_chunks][W] and the per-query row counts.
+struct InterleavePlan {
+  int cap = 0;
+  size_t route = 0, rows = 0, count = 0, bytes = 0;
+};
+
+InterleavePlan plan_interleave(const msa_memory *mem, int B, int T, int k) {
+  InterleavePlan p;
+  p.cap = k * mem->max_doc_chunks;
+  const size_t W = static_cast<size_t>(mem->H_r) * mem->d_r;
+  p.route = 0;
+  const size_t rb = round256(plan_route(mem, B, std::max(T, p.cap), k).bytes);
+  p.rows = rb;
+  p.count = p.rows + round256(static_cast<size_t>(B) * p.cap * W * elem_size(mem->dtype));
+  p.bytes = p.count + round256(static_cast<size_t>(B) * 4);
+  return p;
+}
+
+size_t msa_interleave_workspace_size(const msa_memory *mem, int32_t batch, int32_t tokens,
+                                     int32_t k) {
+  if (!mem || batch < 1 || tokens < 1 || k < 1) return 0;
+  return plan_interleave(mem, batch, tokens, k).bytes;
+}
+
+msa_status msa_interleave(const msa_memory *mem, const void *router_keys, const void *Qr,
+                          int32_t batch, int32_t tokens, int32_t k, int32_t rounds, float *state,
+                          uint8_t *taken, int32_t *ids, float *scores, void *workspace,
+                          size_t workspace_bytes, msa_stream stream) {
+  if (!mem || !router_keys || !Qr || !state || !taken || !ids || !scores)
+    return fail(MSA_ERR_INVALID_ARG, "null argument");
+  if (batch < 1 || tokens < 1 || rounds < 1 || k < 1 || k > mem->n_docs || k > msa::kMaxTopK)
+    return fail(MSA_ERR_INVALID_ARG, "bad batch, tokens, rounds or k");
+  const InterleavePlan plan = plan_interleave(mem, batch, tokens, k);
+  if (!workspace || workspace_bytes < plan.bytes)
+    return fail(MSA_ERR_INVALID_ARG, "workspace too small: %zu < %zu", workspace_bytes, plan.bytes);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  void *rows = ws + plan.rows;
+  int32_t *count = reinterpret_cast<int32_t *>(ws + plan.count);
+  const int W = mem->H_r * mem->d_r;
+  const int64_t nd = static_cast<int64_t>(batch) * mem->n_docs;
+  msa_status r = msa_route_reset(state, nd, stream);
+  if (r != MSA_OK) return r;
+  MSA_CUDA(cudaMemsetAsync(taken, 0, static_cast<size_t>(nd), st));
+  const void *q = Qr;
+  int T = tokens;
+  std::vector<int32_t> h_count(batch);
+  for (int round = 0; round < rounds; ++round) {
+    int32_t *ids_r = ids + static_cast<int64_t>(round) * batch * k;
+    float *sc_r = scores + static_cast<int64_t>(round) * batch * k;
+    r = route_impl(mem, router_keys, q, batch, T, k, taken, state, ids_r, sc_r, ws, plan.rows, st,
+                   q == Qr ? T : plan.cap);
+    if (r != MSA_OK) return r;
+    if (round + 1 == rounds) break;
+    if (mem->dtype == MSA_BF16) {
+      msa::gather_rows_kernel<__nv_bfloat16><<<batch, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16 *>(router_keys), ids_r, k, mem->d_doc_chunk_off,
+          mem->n_docs, W, static_cast<__nv_bfloat16 *>(rows), plan.cap, taken, count);
+    } else {
+      msa::gather_rows_kernel<float><<<batch, 256, 0, st>>>(
+          static_cast<const float *>(router_keys), ids_r, k, mem->d_doc_chunk_off, mem->n_docs, W,
+          static_cast<float *>(rows), plan.cap, taken, count);
+    }
+    MSA_LAUNCHED("gather_rows_kernel");
+    MSA_CUDA(cudaMemcpyAsync(h_count.data(), count, batch * sizeof(int32_t),
+                             cudaMemcpyDeviceToHost, st));
+    MSA_CUDA(cudaStreamSynchronize(st));
+    int T_next = 0;
+    for (int b = 0; b < batch; ++b) T_next = std::max(T_next, static_cast<int>(h_count[b]));
+    if (T_next == 0) T_next = 1;  // nothing retrieved: route one (zero) row
+    if (mem->dtype == MSA_BF16) {
+      msa::pad_rows_kernel<__nv_bfloat16><<<batch, 256, 0, st>>>(
+          static_cast<__nv_bfloat16 *>(rows), plan.cap, W, count, T_next);
+    } else {
+      msa::pad_rows_kernel<float><<<batch, 256, 0, st>>>(static_cast<float *>(rows), plan.cap, W,
+                                                          count, T_next);
+    }
+    MSA_LAUNCHED("pad_rows_kernel");
+    // rows[b] holds cap rows; the route reads the first T_next of each (row pitch cap)
+    q = rows;
+    T = T_next;
+  }
+  return MSA_OK;
 }
 
 msa_status msa_device_error(uint32_t *bits, msa_stream stream) {

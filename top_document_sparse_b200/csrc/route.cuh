@@ -16,13 +16,16 @@ namespace msa {
 
 // Q_hat[r][h][:] = Q_r[r][h][:] / max(|Q_r[r][h]|, eps).  One CTA per row;
 // thread i owns 4 elements; the d_r/4 threads of a head form an aligned group.
+// Row r = b * T + t of the output reads input row b * pitch + t.
 template <typename T>
-__global__ void qnorm_kernel(const T *__restrict__ Qr, int W, int d_r, T *__restrict__ out) {
+__global__ void qnorm_kernel(const T *__restrict__ Qr, int W, int d_r, int T_tok, int pitch,
+                             T *__restrict__ out) {
   const int64_t r = blockIdx.x;
+  const int64_t src_row = (r / T_tok) * pitch + r % T_tok;
   const int e0 = threadIdx.x * 4;
   const bool active = e0 < W;
   float v[4] = {0.f, 0.f, 0.f, 0.f};
-  if (active) load4(Qr + r * W + e0, v);
+  if (active) load4(Qr + src_row * W + e0, v);
   float ss = 0.0f;
 #pragma unroll
   for (int e = 0; e < 4; ++e) ss = fmaf(v[e], v[e], ss);
@@ -171,6 +174,62 @@ route_simt_kernel(const T *__restrict__ Khat, const T *__restrict__ Qhat, int64_
   query_span(r0, NR, T_tok, b0, q_lo, q_hi);
   epi_doc_max(S, 33, MC, QB, b0, docs, prev_doc, next_doc, q_lo, q_hi, n_docs, state, segs, tid,
               256);
+}
+
+// ---------------------------------------------------------------- interleave
+// Memory Interleave (Evermind summary sec. 4C, b-lab.team item 3): the
+// documents retrieved in a round become part of the next round's query.
+// gather_rows_kernel, grid (B): rows[b][0..n_b) = the unit router rows of
+// every chunk of ids[b][0..k), in rank order (n_b <= cap); taken[b][id] = 1;
+// count[b] = n_b.  pad_rows_kernel then copies row 0 of each query over
+// rows[b][n_b..T) so every query has T rows (a repeated row leaves the max
+// over rows unchanged).
+template <typename T>
+__global__ void gather_rows_kernel(const T *__restrict__ keys, const int32_t *__restrict__ ids,
+                                   int k, const int64_t *__restrict__ doc_chunk_off, int n_docs,
+                                   int W, T *__restrict__ rows, int cap,
+                                   uint8_t *__restrict__ taken, int32_t *__restrict__ count) {
+  const int b = blockIdx.x;
+  __shared__ int s_pos;
+  if (threadIdx.x == 0) s_pos = 0;
+  __syncthreads();
+  for (int r = 0; r < k; ++r) {
+    const int d = ids[static_cast<int64_t>(b) * k + r];
+    if (d < 0 || d >= n_docs) continue;
+    if (threadIdx.x == 0) taken[static_cast<int64_t>(b) * n_docs + d] = 1;
+    const int64_t c0 = doc_chunk_off[d], c1 = doc_chunk_off[d + 1];
+    const int pos = s_pos;
+    const int n = static_cast<int>(min(c1 - c0, static_cast<int64_t>(cap - pos)));
+    const int64_t total = static_cast<int64_t>(n) * W / 4;  // 4-element vectors
+    T *dst = rows + (static_cast<int64_t>(b) * cap + pos) * W;
+    const T *src = keys + c0 * W;
+    for (int64_t i = threadIdx.x; i < total; i += blockDim.x) {
+      float v[4];
+      load4(src + 4 * i, v);
+      store4(dst + 4 * i, v);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) s_pos = pos + n;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) count[b] = s_pos;
+}
+
+template <typename T>
+__global__ void pad_rows_kernel(T *__restrict__ rows, int cap, int W,
+                                const int32_t *__restrict__ count, int T_rows) {
+  const int b = blockIdx.x;
+  const int n = count[b];
+  if (n <= 0 || n >= T_rows) return;
+  const T *src = rows + static_cast<int64_t>(b) * cap * W;
+  const int64_t per = W / 4;
+  const int64_t total = static_cast<int64_t>(T_rows - n) * per;
+  for (int64_t i = threadIdx.x; i < total; i += blockDim.x) {
+    const int64_t row = n + i / per, e = (i % per) * 4;
+    float v[4];
+    load4(src + e, v);
+    store4(rows + (static_cast<int64_t>(b) * cap + row) * W + e, v);
+  }
 }
 
 }  // namespace msa

@@ -87,6 +87,9 @@ SIGNATURES = {
                                                  _P, _P, _P, _I32, _I32, _P, _P, _SZ, _P]),
     "msa_step_host": (ctypes.c_int, [_P, _P, _P, ctypes.POINTER(DecodeState), _P, _P, _P, _P, _P,
                                      _P, _P]),
+    "msa_interleave_workspace_size": (_SZ, [_P, _I32, _I32, _I32]),
+    "msa_interleave": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ,
+                                      _P]),
     "msa_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "msa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "msa_last_error": (ctypes.c_char_p, []),
@@ -237,6 +240,21 @@ class Memory:
                                              _ptr(Q), _ptr(K_new), _ptr(V_new), _ptr(K_cache),
                                              _ptr(V_cache), _ptr(cache_len), K_cache.shape[1],
                                              pos_offset, _ptr(O), _stream(stream)))
+
+    def interleave(self, router_keys, Qr, k: int, rounds: int, stream=None):
+        """Memory Interleave rounds (msa_interleave): returns (ids [rounds][B][k], scores,
+        state [B][n_docs], taken [B][n_docs])."""
+        B, T = Qr.shape[0], Qr.shape[1]
+        dev = Qr.device
+        state = torch.empty(B, self.n_docs, dtype=torch.float32, device=dev)
+        taken = torch.empty(B, self.n_docs, dtype=torch.uint8, device=dev)
+        ids = torch.empty(rounds, B, k, dtype=torch.int32, device=dev)
+        scores = torch.empty(rounds, B, k, dtype=torch.float32, device=dev)
+        ws = workspace(_lib.msa_interleave_workspace_size(self.handle, B, T, k), dev)
+        _check(_lib.msa_interleave(self.handle, _ptr(router_keys), _ptr(Qr), B, T, k, rounds,
+                                   _ptr(state), _ptr(taken), _ptr(ids), _ptr(scores), _ptr(ws),
+                                   ws.numel(), _stream(stream)))
+        return ids, scores, state, taken
 
     def step_workspace_size(self, batch: int, k: int, n_q_heads: int) -> int:
         return _lib.msa_step_workspace_size(self.handle, batch, k, n_q_heads)
