@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-100m", action="store_true", help="skip the 100M-token host-tier run")
+    ap.add_argument("--no-interleave", action="store_true", help="skip the Memory Interleave run")
     return ap.parse_args()
 
 
@@ -83,13 +84,21 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
+    """The slowest rank's time: every rank's clock covers the same barrier-bracketed region."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(local_ms: float, units_per_rank: int, world: int, device="cuda") -> tuple:
+    """(max-over-ranks milliseconds, units per second of the whole job): every rank processes
+    units_per_rank units (weak scaling: replicas with their own memory and batch)."""
+    ms = max_over_ranks(local_ms, world, device)
+    return ms, world * units_per_rank / (ms / 1e3)
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -288,7 +297,7 @@ def run_gpu(args, w, world, rank, local):
         e1.record(cur)
         torch.cuda.synchronize()
     barrier(world)
-    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    ms, value = whole_job_rate(e0.elapsed_time(e1), K, world)
     ms_per_step = ms / K
     assert msa.device_error() == 0
 
@@ -392,17 +401,17 @@ def run_gpu(args, w, world, rank, local):
     }
     dom = max(kernels, key=lambda n: kernels[n]["ms_per_call"])
     traffic = None
-    tr_path = os.path.join(ROOT, "profiles", "traffic.json")
+    tr_path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if os.path.exists(tr_path):
         with open(tr_path) as f:
-            traffic = json.load(f).get(w.name, {}).get(dom)
+            traffic = json.load(f).get(w.name, {}).get(dom, {}).get("bytes_per_launch")
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["achieved_gbs"],
                 "peak": hbm, "unit": "GB/s", "frac": kernels[dom]["frac"], "traffic": traffic,
                 "peak_source": peak_kind}
     ceiling_ms = step_bytes / (hbm * 1e9) * 1e3
     res = {
         "metric": METRIC,
-        "value": round(world * K / (ms / 1e3), 2),
+        "value": round(value, 2),
         "unit": "steps/s",
         "n_gpus": world, "steps": K, "warmup": Wm,
         "ms_per_step": round(ms_per_step, 5),
@@ -596,6 +605,58 @@ def run_mem100m(w, msa, episodes=4, seed=4321):
     return res
 
 
+# ---------------------------------------------------------------------------- interleave
+def run_interleave(w, msa, seed=777, reps=3):
+    """The Memory Interleave workload: 1M tokens of lognormal-length documents, 256 queries of 256
+    tokens, 3 rounds of routing with a planted 3-hop chain per query, then one attention of the
+    query block over every retrieved document."""
+    dev = "cuda"
+    off = inputs.doc_offsets(w, seed)
+    dt = inputs.torch_dtype(w.dtype)
+    B, T, k, R = w.batch, w.query_tokens, w.top_k, w.rounds
+    K, V, Kr = inputs.raw_memory(w, int(off[-1]), seed, dev)
+    Qr, Q, Kn, Vn = inputs.queries(w, B, T, seed + 1, dev)
+    chain = inputs.plant_chain(w, Kr, Qr, off, hops=R, seed=seed + 2)
+    mem = msa.Memory(off, w.chunk_len, w.n_kv_heads, w.head_dim, w.n_router_heads, w.router_dim,
+                     dt, w.rope_theta, R * k + T)
+    rk, ct = mem.new_router_keys(), mem.new_content()
+    mem.encode(0, mem.n_docs, K, V, Kr, rk, ct)
+    del K, V, Kr
+    torch.cuda.synchronize()
+    ids, scores, _, _ = mem.interleave(rk, Qr, k, R)  # warm-up
+    torch.cuda.synchronize()
+    t = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        ids, scores, _, _ = mem.interleave(rk, Qr, k, R)
+        b.record()
+        torch.cuda.synchronize()
+        t.append(a.elapsed_time(b))
+    got = ids.cpu().numpy()
+    hop_rate = [float(np.mean([chain[q, r] in got[r, q] for q in range(B)])) for r in range(R)]
+    # the sparse generation step over the R * k retrieved documents
+    ctx_ids = ids.permute(1, 0, 2).reshape(B, R * k).contiguous()
+    cap = T
+    Kc = torch.zeros(B, cap, w.n_kv_heads, w.head_dim, dtype=dt, device=dev)
+    Vc = torch.zeros_like(Kc)
+    clen = torch.zeros(B, dtype=torch.int32, device=dev)
+    O = torch.empty(B, T, w.n_q_heads, w.head_dim, dtype=dt, device=dev)
+    ws = msa.workspace(mem.attend_workspace_size(B, T, R * k, w.n_q_heads))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    mem.sparse_attend(ct, ctx_ids, Q, Kn, Vn, Kc, Vc, clen, R * k, O, ws)
+    b.record()
+    torch.cuda.synchronize()
+    return {"workload": w.name, "n_docs": mem.n_docs, "memory_tokens": int(off[-1]),
+            "chunks": int(mem.n_chunks), "batch": B, "query_tokens": T, "top_k": k, "rounds": R,
+            "interleave_ms": round(statistics.median(t), 3),
+            "queries_per_s": round(B / (statistics.median(t) * 1e-3), 1),
+            "hop_retrieved_rate": hop_rate,
+            "final_attend_ms": round(a.elapsed_time(b), 3),
+            "max_doc_chunks": int(mem.info.max_doc_chunks)}
+
+
 # ---------------------------------------------------------------------------- CPU baseline
 class OracleSample:
     """The fp64 oracle on a bounded sample of the workload's decode step: one decode token for a
@@ -706,6 +767,20 @@ def main():
         from top_document_sparse_b200 import msa
         torch.cuda.empty_cache()
         res["mem100m"] = run_mem100m(WORKLOADS["mem100m_bf16"], msa)
+        rs = res["mem100m"]["route_score"]
+        tr = None
+        tr_path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+        if os.path.exists(tr_path):
+            with open(tr_path) as f:
+                tr = json.load(f).get("mem100m_bf16", {}).get("route", {}).get("bytes_per_launch")
+        res["route_score_roofline"] = {
+            "bound": "hbm", "kernel": "route (msa_route call: qnorm + route_tc + top-k)",
+            "workload": "mem100m_bf16", "achieved": rs["achieved_gbs"], "peak": rs["peak"],
+            "unit": "GB/s", "frac": rs["frac"], "traffic": tr, "peak_source": "measured"}
+    if not args.no_interleave and world == 1:
+        from top_document_sparse_b200 import msa
+        torch.cuda.empty_cache()
+        res["interleave"] = run_interleave(WORKLOADS["interleave_bf16"], msa)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:

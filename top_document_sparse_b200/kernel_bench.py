@@ -1,0 +1,112 @@
+"""Per-stage timing of the MSA hot path at a workload's sizes (one routed layer, one decode token).
+
+    python -m top_document_sparse_b200.kernel_bench [--workload mem1m_bf16] [--stage all]
+                                                    [--reps 20]
+
+Stages: ``route`` (msa_route: query normalisation, route score, top-k), ``topk`` (msa_route with
+no query rows), ``attend`` (msa_sparse_attend of one token over k retrieved documents plus the
+local cache).  The router keys are random unit vectors and the pooled content random bf16, so
+no encode pass is needed.  Calls are captured in a CUDA graph and timed with CUDA events; each
+call reads more than the 126 MB L2 only for memories of 64K+ chunks, so small workloads report
+L2-warm figures (printed as "l2_warm").  Used for the ncu captures summarised under profiles/.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import numpy as np
+import torch
+
+from . import msa
+from .inputs import doc_offsets
+from .workloads import WORKLOADS
+
+
+def _graph_time(fn, reps):
+    s = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(reps):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps * 1e3  # us per call
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="mem1m_bf16")
+    ap.add_argument("--stage", default="all", choices=["all", "route", "topk", "attend"])
+    ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--seed", type=int, default=0)
+    a = ap.parse_args(argv)
+    w = WORKLOADS[a.workload]
+    torch.cuda.set_device(0)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(a.seed)
+    off = doc_offsets(w, a.seed)
+    B, k, H_q, D, H_kv = w.batch, w.top_k, w.n_q_heads, w.head_dim, w.n_kv_heads
+    cap = w.query_tokens + max(w.decode_steps, 1)
+    mem = msa.Memory(off, w.chunk_len, H_kv, D, w.n_router_heads, w.router_dim, torch.bfloat16,
+                     w.rope_theta, k + cap)
+    W = w.n_router_heads * w.router_dim
+    out = {"workload": w.name, "chunks": int(mem.n_chunks), "batch": B, "top_k": k,
+           "l2_warm": mem.n_chunks * W * 2 < (126 << 20)}
+    if a.stage in ("all", "route", "topk"):
+        rk = torch.randn(mem.n_chunks, w.n_router_heads, w.router_dim, device="cuda",
+                         generator=gen)
+        rk = (rk / rk.norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+        Qr = torch.randn(B, 1, w.n_router_heads, w.router_dim, device="cuda",
+                         generator=gen).to(torch.bfloat16)
+        st = torch.full((B, mem.n_docs), float("-inf"), device="cuda")
+        ids = torch.zeros(B, k, dtype=torch.int32, device="cuda")
+        sc = torch.zeros(B, k, device="cuda")
+        ws = msa.workspace(mem.route_workspace_size(B, 1, k))
+        byts = mem.n_chunks * W * 2 + 2 * B * mem.n_docs * 4
+        if a.stage in ("all", "route"):
+            t = _graph_time(lambda: mem.route(rk, Qr, k, st, ids, sc, ws), a.reps)
+            out["route_us"] = round(t, 2)
+            out["route_gbs"] = round(byts / (t * 1e-6) / 1e9, 1)
+        if a.stage in ("all", "topk"):
+            out["topk_us"] = round(_graph_time(lambda: mem.route(None, None, k, st, ids, sc, ws),
+                                               a.reps), 2)
+        del rk
+    if a.stage in ("all", "attend"):
+        ct = torch.randn(mem.n_chunks, 2, H_kv, D, device="cuda", generator=gen).to(torch.bfloat16)
+        ids = torch.from_numpy(np.stack([np.random.default_rng(b).choice(mem.n_docs, k, replace=False)
+                                         for b in range(B)]).astype(np.int32)).cuda()
+        Kc = torch.randn(B, cap, H_kv, D, device="cuda", generator=gen).to(torch.bfloat16)
+        Vc = torch.randn(B, cap, H_kv, D, device="cuda", generator=gen).to(torch.bfloat16)
+        Q = torch.randn(B, 1, H_q, D, device="cuda", generator=gen).to(torch.bfloat16)
+        Kn = torch.randn(B, 1, H_kv, D, device="cuda", generator=gen).to(torch.bfloat16)
+        O = torch.empty_like(Q)
+        L0 = w.query_tokens + max(w.decode_steps, 1) // 2
+        clen = torch.full((B,), L0, dtype=torch.int32, device="cuda")
+        ws = msa.workspace(mem.attend_workspace_size(B, 1, k, H_q))
+
+        def att():
+            clen.fill_(L0)
+            mem.sparse_attend(ct, ids, Q, Kn, Kn, Kc, Vc, clen, k, O, ws)
+
+        t = _graph_time(att, a.reps)
+        n_mem = int(sum(mem.doc_chunk_offsets[d + 1] - mem.doc_chunk_offsets[d]
+                        for d in ids.cpu().numpy().ravel()))
+        byts = (n_mem + B * (L0 + 1)) * H_kv * 2 * D * 2
+        out["attend_us"] = round(t, 2)
+        out["attend_gbs"] = round(byts / (t * 1e-6) / 1e9, 1)
+    out["device_error"] = msa.device_error()
+    print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    main()
