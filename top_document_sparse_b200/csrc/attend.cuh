@@ -14,6 +14,8 @@
 //                         online softmax; the GQA group's heads are the M rows
 //   attend_combine_kernel merge context splits (log-sum-exp) and advance
 //                         cache_len
+// For a one-token call (decode) the attention kernel appends the new row
+// itself; longer calls run append_kernel first.
 #pragma once
 #include "common.cuh"
 #include "ptx.cuh"
@@ -234,11 +236,12 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
                   int k, const int64_t *__restrict__ doc_chunk_off, int n_docs,
                   const int32_t *__restrict__ slots, int slot_chunks, int H_kv,
                   const __nv_bfloat16 *__restrict__ Q, int T_tok,
-                  const __nv_bfloat16 *__restrict__ K_cache,
-                  const __nv_bfloat16 *__restrict__ V_cache, const int32_t *__restrict__ cache_len,
-                  int cap, int pos_offset, const float2 *__restrict__ rope, float scale_log2,
-                  int n_split, int table_cap, __nv_bfloat16 *__restrict__ O,
-                  float *__restrict__ part_o, float *__restrict__ part_ml) {
+                  __nv_bfloat16 *__restrict__ K_cache, __nv_bfloat16 *__restrict__ V_cache,
+                  const __nv_bfloat16 *__restrict__ K_new, const __nv_bfloat16 *__restrict__ V_new,
+                  const int32_t *__restrict__ cache_len, int cap, int pos_offset,
+                  const float2 *__restrict__ rope, float scale_log2, int n_split, int table_cap,
+                  int fuse_append, __nv_bfloat16 *__restrict__ O, float *__restrict__ part_o,
+                  float *__restrict__ part_ml) {
   constexpr int CPR = D / 8;  // 16-byte chunks per row
   using Sm = AttSmem<D>;
   extern __shared__ __align__(128) uint8_t sm[];
@@ -257,14 +260,38 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
                                       slots ? slots + static_cast<int64_t>(b) * k : nullptr,
                                       slot_chunks, table, pre, base, table_cap);
   const int j = cache_len[b] + i;
-  const bool overflow = j >= cap;
+  const bool overflow = j >= cap || j < 0;
   const int n_ctx = overflow ? 0 : n_mem + j + 1;
   int per = (n_ctx + n_split - 1) / n_split;
   per = (per + kAttRows - 1) / kAttRows * kAttRows;
   const int x0 = split * per;
   const int x1 = min(n_ctx, x0 + per);
-
   const int64_t kv = static_cast<int64_t>(H_kv) * D;
+  if (fuse_append) {
+    // one-token call: the CTA whose range holds the new row (context row
+    // n_mem + j) rotates K_new at pos_offset + j and writes K and V to the
+    // cache before any of its copies can read that row
+    if (overflow) {
+      if (threadIdx.x == 0 && g == 0 && split == 0) raise_device_error(MSA_DEVERR_CACHE_OVERFLOW);
+    } else if (x0 <= n_mem + j && n_mem + j < x1) {
+      const int half = D / 2;
+      const int64_t src = static_cast<int64_t>(b) * kv + g * D;
+      const int64_t dst = (static_cast<int64_t>(b) * cap + j) * kv + g * D;
+      const float2 *cs = rope + static_cast<int64_t>(pos_offset + j) * half;
+      for (int e = threadIdx.x; e < half; e += blockDim.x) {
+        const float a = __bfloat162float(K_new[src + e]);
+        const float c = __bfloat162float(K_new[src + e + half]);
+        const float2 t = cs[e];
+        K_cache[dst + e] = __float2bfloat16_rn(a * t.x - c * t.y);
+        K_cache[dst + e + half] = __float2bfloat16_rn(c * t.x + a * t.y);
+        V_cache[dst + e] = V_new[src + e];
+        V_cache[dst + e + half] = V_new[src + e + half];
+      }
+      __threadfence();  // the row is read back below through cp.async (L2)
+      __syncthreads();
+    }
+  }
+
   uint8_t *wbuf = ring + warp * Sm::kWarpBytes;
   // issue the loads of the block starting at context row x into stage s
   auto issue = [&](int x, int s) {
@@ -481,11 +508,17 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
 }
 
 // grid (B * T * H_q), block D: merge the context splits.  Partial maxima are
-// in log2 units.  Also advances cache_len[b] by T (one thread per query).
+// in log2 units.  The first block of each query also advances cache_len[b] by
+// T (every attention CTA has read it by now).
 __global__ void attend_combine_kernel(const float *__restrict__ part_o,
                                       const float *__restrict__ part_ml, int n_split, int D,
-                                      __nv_bfloat16 *__restrict__ O) {
+                                      __nv_bfloat16 *__restrict__ O, int32_t *__restrict__ cache_len,
+                                      int rows_per_query, int T_tok, int cap) {
   const int64_t orow = blockIdx.x;
+  if (threadIdx.x == 0 && orow % rows_per_query == 0) {
+    int32_t *cl = cache_len + orow / rows_per_query;
+    *cl = min(*cl + T_tok, cap);
+  }
   const float *ml = part_ml + orow * n_split * 2;
   float M = -INFINITY;
   for (int s = 0; s < n_split; ++s) M = fmaxf(M, ml[2 * s]);

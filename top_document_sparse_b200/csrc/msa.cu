@@ -291,8 +291,8 @@ msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, i
 template <int D, int G>
 msa_status launch_attend_mma(const msa_memory *mem, const void *content, const int32_t *ids,
                              const int32_t *slots, int slot_chunks, int B, int k, int T,
-                             const void *Q, const void *Kc, const void *Vc,
-                             const int32_t *cache_len, int cap, int pos_offset,
+                             const void *Q, const void *K_new, const void *V_new, void *Kc,
+                             void *Vc, int32_t *cache_len, int cap, int pos_offset,
                              const AttendPlan &plan, void *O, void *ws, cudaStream_t st) {
   using Sm = msa::AttSmem<D>;
   const int smem = Sm::bytes(plan.table_cap);
@@ -302,19 +302,26 @@ msa_status launch_attend_mma(const msa_memory *mem, const void *content, const i
   float *part_o = plan.n_split > 1 ? reinterpret_cast<float *>(wsb + plan.part_o) : nullptr;
   float *part_ml = plan.n_split > 1 ? reinterpret_cast<float *>(wsb + plan.part_ml) : nullptr;
   const float scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)) * 1.4426950408889634);
+  const int fuse_append = T == 1 ? 1 : 0;
   dim3 grid(static_cast<unsigned>(B * mem->H_kv), plan.n_split, T);
-  kern<<<grid, 128, smem, st>>>(
+  kern<<<grid, 32 * msa::kAttWarps, smem, st>>>(
       static_cast<const __nv_bfloat16 *>(content), ids, k, mem->d_doc_chunk_off, mem->n_docs, slots,
       slot_chunks, mem->H_kv, static_cast<const __nv_bfloat16 *>(Q), T,
-      static_cast<const __nv_bfloat16 *>(Kc), static_cast<const __nv_bfloat16 *>(Vc), cache_len,
-      cap, pos_offset, mem->d_rope, scale_log2, plan.n_split, plan.table_cap,
-      static_cast<__nv_bfloat16 *>(O), part_o, part_ml);
+      static_cast<__nv_bfloat16 *>(Kc), static_cast<__nv_bfloat16 *>(Vc),
+      static_cast<const __nv_bfloat16 *>(K_new), static_cast<const __nv_bfloat16 *>(V_new),
+      cache_len, cap, pos_offset, mem->d_rope, scale_log2, plan.n_split, plan.table_cap,
+      fuse_append, static_cast<__nv_bfloat16 *>(O), part_o, part_ml);
   MSA_LAUNCHED("attend_mma_kernel");
   if (plan.n_split > 1) {
+    // merge the splits and advance cache_len (every attention CTA has read it)
     msa::attend_combine_kernel<<<static_cast<unsigned>(static_cast<int64_t>(B) * T * mem->H_kv * G),
                                  D, 0, st>>>(part_o, part_ml, plan.n_split, D,
-                                             static_cast<__nv_bfloat16 *>(O));
+                                             static_cast<__nv_bfloat16 *>(O), cache_len,
+                                             T * mem->H_kv * G, T, cap);
     MSA_LAUNCHED("attend_combine_kernel");
+  } else {
+    msa::advance_kernel<<<(B + 255) / 256, 256, 0, st>>>(cache_len, B, T, cap);
+    MSA_LAUNCHED("advance_kernel");
   }
   return MSA_OK;
 }
@@ -322,13 +329,13 @@ msa_status launch_attend_mma(const msa_memory *mem, const void *content, const i
 template <int D>
 msa_status dispatch_group(int G, const msa_memory *mem, const void *content, const int32_t *ids,
                           const int32_t *slots, int slot_chunks, int B, int k, int T,
-                          const void *Q, const void *Kc, const void *Vc, const int32_t *cache_len,
-                          int cap, int pos_offset, const AttendPlan &plan, void *O, void *ws,
-                          cudaStream_t st) {
+                          const void *Q, const void *K_new, const void *V_new, void *Kc, void *Vc,
+                          int32_t *cache_len, int cap, int pos_offset, const AttendPlan &plan,
+                          void *O, void *ws, cudaStream_t st) {
 #define MSA_G(g)                                                                                  \
   case g:                                                                                         \
-    return launch_attend_mma<D, g>(mem, content, ids, slots, slot_chunks, B, k, T, Q, Kc, Vc,     \
-                                   cache_len, cap, pos_offset, plan, O, ws, st);
+    return launch_attend_mma<D, g>(mem, content, ids, slots, slot_chunks, B, k, T, Q, K_new,      \
+                                   V_new, Kc, Vc, cache_len, cap, pos_offset, plan, O, ws, st);
   switch (G) {
     MSA_G(1) MSA_G(2) MSA_G(4) MSA_G(8) MSA_G(16)
     default:
@@ -369,51 +376,49 @@ msa_status attend_impl(const msa_memory *mem, const void *content, const int32_t
   if (ws_bytes < plan.bytes || (plan.bytes > 0 && !ws))
     return fail(MSA_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, plan.bytes);
   const int D = mem->D, H_kv = mem->H_kv;
-  // 1. append the new tokens (K rotated at pos_offset + j)
+  if (mem->dtype == MSA_BF16) {
+    // one token: the attention kernel appends the new row itself; more: append first
+    if (T > 1) {
+      const int athr = round32(H_kv * D / 8);
+      if (athr > 1024) return fail(MSA_ERR_UNSUPPORTED, "n_kv_heads * head_dim too large");
+      msa::append_kernel<__nv_bfloat16><<<B * T, athr, 0, st>>>(
+          static_cast<const __nv_bfloat16 *>(K_new), static_cast<const __nv_bfloat16 *>(V_new), T,
+          H_kv, D, static_cast<__nv_bfloat16 *>(K_cache), static_cast<__nv_bfloat16 *>(V_cache),
+          cache_len, cap, pos_offset, mem->d_rope);
+      MSA_LAUNCHED("append_kernel");
+    }
+    const int G = H_q / H_kv;
+    if (D == 128)
+      return dispatch_group<128>(G, mem, content, ids, slots, slot_chunks, B, k, T, Q, K_new,
+                                 V_new, K_cache, V_cache, cache_len, cap, pos_offset, plan, O, ws,
+                                 st);
+    return dispatch_group<64>(G, mem, content, ids, slots, slot_chunks, B, k, T, Q, K_new, V_new,
+                              K_cache, V_cache, cache_len, cap, pos_offset, plan, O, ws, st);
+  }
+  // fp32: append, attention, advance
+  if (H_q > 16) return fail(MSA_ERR_UNSUPPORTED, "fp32 attention supports <= 16 query heads");
   const int athr = round32(H_kv * D / 8);
   if (athr > 1024) return fail(MSA_ERR_UNSUPPORTED, "n_kv_heads * head_dim too large");
-  if (mem->dtype == MSA_BF16) {
-    msa::append_kernel<__nv_bfloat16><<<B * T, athr, 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(K_new), static_cast<const __nv_bfloat16 *>(V_new), T,
-        H_kv, D, static_cast<__nv_bfloat16 *>(K_cache), static_cast<__nv_bfloat16 *>(V_cache),
-        cache_len, cap, pos_offset, mem->d_rope);
-  } else {
-    msa::append_kernel<float><<<B * T, athr, 0, st>>>(
-        static_cast<const float *>(K_new), static_cast<const float *>(V_new), T, H_kv, D,
-        static_cast<float *>(K_cache), static_cast<float *>(V_cache), cache_len, cap, pos_offset,
-        mem->d_rope);
-  }
+  msa::append_kernel<float><<<B * T, athr, 0, st>>>(
+      static_cast<const float *>(K_new), static_cast<const float *>(V_new), T, H_kv, D,
+      static_cast<float *>(K_cache), static_cast<float *>(V_cache), cache_len, cap, pos_offset,
+      mem->d_rope);
   MSA_LAUNCHED("append_kernel");
-  // 2. attention over [memory rows | causal local rows]
-  const int G = H_q / H_kv;
-  msa_status s = MSA_OK;
-  if (mem->dtype == MSA_BF16) {
-    if (D == 128)
-      s = dispatch_group<128>(G, mem, content, ids, slots, slot_chunks, B, k, T, Q, K_cache,
-                              V_cache, cache_len, cap, pos_offset, plan, O, ws, st);
-    else
-      s = dispatch_group<64>(G, mem, content, ids, slots, slot_chunks, B, k, T, Q, K_cache,
-                             V_cache, cache_len, cap, pos_offset, plan, O, ws, st);
-  } else {
-    if (H_q > 16) return fail(MSA_ERR_UNSUPPORTED, "fp32 attention supports <= 16 query heads");
-    const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
-    const int thr = H_q * 32;
-    if (D == 128)
-      msa::attend_simt_kernel<float, 128><<<B * T, thr, 0, st>>>(
-          static_cast<const float *>(content), ids, k, mem->d_doc_chunk_off, mem->n_docs, slots,
-          slot_chunks, H_kv, H_q, static_cast<const float *>(Q), T,
-          static_cast<const float *>(K_cache), static_cast<const float *>(V_cache), cache_len, cap,
-          pos_offset, mem->d_rope, scale, static_cast<float *>(O));
-    else
-      msa::attend_simt_kernel<float, 64><<<B * T, thr, 0, st>>>(
-          static_cast<const float *>(content), ids, k, mem->d_doc_chunk_off, mem->n_docs, slots,
-          slot_chunks, H_kv, H_q, static_cast<const float *>(Q), T,
-          static_cast<const float *>(K_cache), static_cast<const float *>(V_cache), cache_len, cap,
-          pos_offset, mem->d_rope, scale, static_cast<float *>(O));
-    MSA_LAUNCHED("attend_simt_kernel");
-  }
-  if (s != MSA_OK) return s;
-  // 3. the cache now holds T more rows
+  const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  const int thr = H_q * 32;
+  if (D == 128)
+    msa::attend_simt_kernel<float, 128><<<B * T, thr, 0, st>>>(
+        static_cast<const float *>(content), ids, k, mem->d_doc_chunk_off, mem->n_docs, slots,
+        slot_chunks, H_kv, H_q, static_cast<const float *>(Q), T,
+        static_cast<const float *>(K_cache), static_cast<const float *>(V_cache), cache_len, cap,
+        pos_offset, mem->d_rope, scale, static_cast<float *>(O));
+  else
+    msa::attend_simt_kernel<float, 64><<<B * T, thr, 0, st>>>(
+        static_cast<const float *>(content), ids, k, mem->d_doc_chunk_off, mem->n_docs, slots,
+        slot_chunks, H_kv, H_q, static_cast<const float *>(Q), T,
+        static_cast<const float *>(K_cache), static_cast<const float *>(V_cache), cache_len, cap,
+        pos_offset, mem->d_rope, scale, static_cast<float *>(O));
+  MSA_LAUNCHED("attend_simt_kernel");
   msa::advance_kernel<<<(B + 255) / 256, 256, 0, st>>>(cache_len, B, T, cap);
   MSA_LAUNCHED("advance_kernel");
   return MSA_OK;
