@@ -230,9 +230,9 @@ MSA_API msa_status msa_sparse_attend(const msa_memory *mem, const void *content,
  * Arguments are those of msa_sparse_attend without `workspace` and
  * `workspace_bytes`; the caller still passes every input and output buffer.
  * The call allocates nothing.  Its scratch (the partial results of the split
- * attention context) lives in one fixed device array of 8 MiB (8388608 bytes)
+ * attention context) lives in one fixed device array of 4 MiB (4194304 bytes)
  * inside the library; every GPU that loads the library holds that array until
- * the process exits.  A call whose scratch would exceed 8 MiB (the size
+ * the process exits.  A call whose scratch would exceed 4 MiB (the size
  * msa_attend_workspace_size reports for the same arguments, with
  * cache_capacity in place of max_local_position) is rejected with
  * MSA_ERR_UNSUPPORTED and enqueues nothing.
@@ -375,6 +375,11 @@ MSA_API msa_status msa_device_error(uint32_t *bits, msa_stream stream);
 
 MSA_API const char *msa_status_string(msa_status s);
 MSA_API const char *msa_last_error(void);
+/* Number of kernels this library has enqueued from this process so far, over
+ * all threads and devices.  A launch made while a stream is being captured
+ * into a CUDA graph counts once, at capture, not per replay.  No counterpart
+ * in the method: it lets a caller count the kernels of a timed region. */
+MSA_API uint64_t msa_launch_count(void);
 /* Library version as major*10000 + minor*100 + patch. */
 MSA_API int32_t msa_version(void);
 

@@ -1,6 +1,6 @@
 """msa_sparse_attend_static: the attention entry point for callers that cannot allocate device
 memory (for example a plugin inside a host engine that reserved the whole device budget up front).
-It takes no workspace; its scratch is a fixed 8 MiB array inside the library.  This file runs last
+It takes no workspace; its scratch is a fixed 4 MiB array inside the library.  This file runs last
 (pytest collects it after the others) and must pass both alone in a fresh process and after the
 rest of the suite: two calls in a row must give the same outputs and the same local cache as the
 workspace entry point on the same inputs."""
@@ -52,17 +52,22 @@ def test_static_scratch_attention_matches_workspace_entry_point():
 
 
 def test_static_scratch_rejects_calls_beyond_its_size():
-    """A call whose split-context scratch would exceed the 8 MiB array is refused on the host
-    and enqueues nothing (every buffer below is sized for the call all the same)."""
+    """A call whose split-context scratch would exceed the 4 MiB array is refused on the host
+    and enqueues nothing (every buffer below is sized for the call all the same).  The split
+    count aims at about three CTAs per SM, so the largest scratch comes from a call with just
+    fewer (query, token, kv head) CTAs than that and 16 query heads per kv head."""
     from top_document_sparse_b200 import msa
-    w = small_workload(n_q_heads=128, n_kv_heads=8, head_dim=128, batch=8, top_k=4, n_docs=12,
-                       doc_len=448)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    B, k, H_kv, D, cap = 4, 4, 1, 128, 512
+    H_q = 16 * H_kv
+    T = (3 * sms - 1) // (B * H_kv)            # B * T * H_kv just under 3 CTAs per SM: 2 splits
+    w = small_workload(n_q_heads=H_q, n_kv_heads=H_kv, head_dim=D, batch=B, top_k=k,
+                       n_docs=12, doc_len=448)
     inp = memory_inputs(w, seed=911)
-    B, T, k, H_q, H_kv, D, cap = 8, 4, 4, 128, 8, 128, 512
     mem = msa.Memory(inp["off"], w.chunk_len, H_kv, D, w.n_router_heads, w.router_dim,
                      torch.bfloat16, w.rope_theta, k + cap)
     need = mem.attend_workspace_size(B, T, k, H_q)
-    assert need > (8 << 20)
+    assert need > (4 << 20)
     ct = torch.zeros(mem.n_chunks, 2, H_kv, D, dtype=torch.bfloat16, device="cuda")
     Q = torch.zeros(B, T, H_q, D, dtype=torch.bfloat16, device="cuda")
     Kn = torch.zeros(B, T, H_kv, D, dtype=torch.bfloat16, device="cuda")

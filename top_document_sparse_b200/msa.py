@@ -94,6 +94,7 @@ SIGNATURES = {
     "msa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "msa_last_error": (ctypes.c_char_p, []),
     "msa_version": (ctypes.c_int32, []),
+    "msa_launch_count": (ctypes.c_uint64, []),
 }
 
 
@@ -116,6 +117,11 @@ _lib = load_library()
 
 def lib() -> ctypes.CDLL:
     return _lib
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued (graph captures count once, at capture)."""
+    return int(_lib.msa_launch_count())
 
 
 def _check(status: int):
