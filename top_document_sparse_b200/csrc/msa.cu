@@ -192,10 +192,13 @@ RoutePlan plan_route(const msa_memory *mem, int B, int T, int k) {
   return p;
 }
 
-template <int NT>
+// NT = 64 query rows stream their feature slices with the key slices (a
+// resident 64-row tile would leave only four ring stages); narrower tiles
+// stay resident.
+template <int NT, bool QS = (NT >= 64)>
 msa_status launch_route_tc(const msa_memory *mem, const void *keys, const void *qhat, int R, int T,
                            float *state, cudaStream_t st) {
-  using L = msa::RouteTcLayout<NT>;
+  using L = msa::RouteTcLayout<NT, QS>;
   const int W = mem->H_r * mem->d_r;
   CUtensorMap tmK, tmQ;
   msa_status s = make_map_bf16(&tmK, keys, mem->n_chunks, W, L::kTileC);
@@ -208,7 +211,7 @@ msa_status launch_route_tc(const msa_memory *mem, const void *keys, const void *
   const size_t smem = L::bytes(W, stages);
   if (smem + 256 > static_cast<size_t>(maxs))
     return fail(MSA_ERR_UNSUPPORTED, "router width %d needs %zu B of shared memory", W, smem);
-  auto kern = msa::route_tc_kernel<NT>;
+  auto kern = msa::route_tc_kernel<NT, QS>;
   MSA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const int n_ct = static_cast<int>((mem->n_chunks + L::kTileC - 1) / L::kTileC);
   const int n_rt = (R + NT - 1) / NT;

@@ -64,8 +64,8 @@ __device__ __forceinline__ void epi_token_max(float *S, int ldS, int MC, int NR,
 
 // Stage 2 (all nthr threads must call it: it holds named barrier 2): for each
 // (document run inside the tile, query), max over the run's
-// chunks, then max-merge into state.  `segs` (shared, >= MC + 1 ints) receives
-// the run starts.  A run whose document lies wholly inside the chunk tile, for
+// chunks (written over the run's first row of S), then max-merge into state.
+// `segs` (shared, >= MC + 1 ints) receives the run starts.  A run whose document lies wholly inside the chunk tile, for
 // a query whose rows lie wholly inside the row tile, has this CTA as its only
 // writer during the call: it is merged with a plain load / max / store
 // (consecutive threads take consecutive documents, so the accesses coalesce).
@@ -74,7 +74,7 @@ __device__ __forceinline__ void epi_token_max(float *S, int ldS, int MC, int NR,
 //   prev_doc / next_doc: document of the chunk just before / after the tile
 //   (-1 at the memory's ends); q_lo / q_hi: the queries whose rows are all
 //   inside the row tile are [q_lo, q_hi) (relative to b0).
-__device__ __forceinline__ void epi_doc_max(const float *S, int ldS, int MC, int QB, int64_t b0,
+__device__ __forceinline__ void epi_doc_max(float *S, int ldS, int MC, int QB, int64_t b0,
                                             const int *docs, int prev_doc, int next_doc,
                                             int q_lo, int q_hi, int n_docs, float *state,
                                             int *segs, int tid, int nthr, bool write = true) {
@@ -96,19 +96,60 @@ __device__ __forceinline__ void epi_doc_max(const float *S, int ldS, int MC, int
   }
   if (tid == 0) segs[n_seg] = MC;
   asm volatile("bar.sync 2, %0;" ::"r"(nthr) : "memory");
+  // Pass A: run maxima in place -- S[segs[g]][q] = max over run g of column q.
+  // Thread t takes column q = t % QB (consecutive lanes, consecutive banks) and
+  // every (nthr / QB)-th run.  (`write` may differ between threads: every
+  // thread still takes the barrier below.)
+  const int cols = QB < nthr ? QB : nthr;
+  const int per_col = nthr / cols;
+  if (write && tid < cols * per_col) {
+    const int q0 = tid % cols;
+    for (int q = q0; q < QB; q += cols)
+      for (int g = tid / cols; g < n_seg; g += per_col) {
+        const int m0 = segs[g], m1 = segs[g + 1];
+        float x = S[m0 * ldS + q];
+        for (int m = m0 + 1; m < m1; ++m) x = fmaxf(x, S[m * ldS + q]);
+        S[m0 * ldS + q] = x;
+      }
+  }
+  asm volatile("bar.sync 2, %0;" ::"r"(nthr) : "memory");
   if (!write) return;  // every thread has passed the barriers above
-  for (int p = tid; p < n_seg * QB; p += nthr) {
-    const int q = p / n_seg, g = p - q * n_seg;
-    const int m0 = segs[g], m1 = segs[g + 1];
-    const int d = docs[m0];
-    float v = S[m0 * ldS + q];
-    for (int m = m0 + 1; m < m1; ++m) v = fmaxf(v, S[m * ldS + q]);
-    float *dst = state + (b0 + q) * n_docs + d;
-    const bool whole_doc = (m0 > 0 || prev_doc != d) && (m1 < MC || next_doc != d);
-    if (whole_doc && q >= q_lo && q < q_hi) {
-      *dst = fmaxf(*dst, v);
-    } else {
-      atomic_max_float(dst, v);
+  // Pass B: merge into state.  Consecutive threads take consecutive documents
+  // of one query (coalesced).  A thread takes up to kBatch pairs and issues all
+  // their state loads before any store: the pairs are distinct state entries
+  // (a document is one run of the tile), so the loads overlap.  A run whose
+  // document lies wholly inside the chunk tile, for a query whose rows lie
+  // wholly inside the row tile, has this CTA as its only writer during the
+  // call (plain load / max / store); the others use an atomic float max.
+  constexpr int kBatch = 8;
+  const int total = n_seg * QB;
+  for (int p0 = tid; p0 < total; p0 += kBatch * nthr) {
+    float v[kBatch], old[kBatch];
+    float *dst[kBatch];
+    bool plain[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int p = p0 + u * nthr;
+      dst[u] = nullptr;
+      plain[u] = false;
+      if (p < total) {
+        const int q = p / n_seg, g = p - q * n_seg;
+        const int m0 = segs[g], m1 = segs[g + 1];
+        const int d = docs[m0];
+        v[u] = S[m0 * ldS + q];
+        dst[u] = state + (b0 + q) * n_docs + d;
+        const bool whole_doc = (m0 > 0 || prev_doc != d) && (m1 < MC || next_doc != d);
+        plain[u] = whole_doc && q >= q_lo && q < q_hi;
+        if (plain[u]) old[u] = *dst[u];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (dst[u] == nullptr) continue;
+      if (plain[u])
+        *dst[u] = fmaxf(old[u], v[u]);
+      else
+        atomic_max_float(dst[u], v[u]);
     }
   }
 }
@@ -166,7 +207,7 @@ route_simt_kernel(const T *__restrict__ Khat, const T *__restrict__ Qhat, int64_
   const int prev_doc = c0 > 0 ? chunk_doc[c0 - 1] : -1;
   const int next_doc = c0 + MC < C ? chunk_doc[c0 + MC] : -1;
   __syncthreads();
-  epi_token_max(S, 33, MC, NR, r0, T_tok, tid, 256);
+  if (T_tok > 1) epi_token_max(S, 33, MC, NR, r0, T_tok, tid, 256);
   __syncthreads();
   const int64_t b0 = r0 / T_tok;
   const int QB = static_cast<int>((r0 + NR - 1) / T_tok - b0 + 1);

@@ -9,7 +9,8 @@
 //
 // Warp roles (192 threads):
 //   warp 4  one lane: TMA producer -- query rows of the row tile (resident,
-//           all W features) and a ring of 64-feature x 128-chunk key slices
+//           all W features; or streamed slice by slice, QS) and a ring of
+//           64-feature x 128-chunk key slices
 //   warp 5  allocates TMEM; one lane issues 4 UMMAs (K = 16 each) per slice
 //           and commits them to the slice's "empty" barrier, then commits
 //           the finished accumulator to "acc full"
@@ -26,27 +27,36 @@
 
 namespace msa {
 
-template <int NT>
+// QS (streamed query): the producer copies the row tile's 64-feature query
+// slice into each ring stage next to the key slice, instead of keeping all W
+// features of the NT query rows resident.  With NT = 64 and W = 1024 the
+// resident rows would take 128 KiB and leave room for only four key slices in
+// flight; streamed, the ring holds about eight (24 KiB) stages.
+template <int NT, bool QS>
 struct RouteTcLayout {
   static constexpr int kTileC = 128;
   static constexpr int kSlice = kTileC * 128;  // 16 KiB: 128 rows x 64 bf16
+  static constexpr int kQSlice = NT * 128;     // NT rows x 64 bf16
+  static constexpr int kStage = kSlice + (QS ? kQSlice : 0);
   static constexpr int kLD = NT + 1;           // epilogue staging row stride (floats)
   static constexpr uint32_t kTmemCols = (2 * NT < 32) ? 32 : 2 * NT;
-  static __host__ __device__ size_t q_bytes(int W) { return static_cast<size_t>(W / 64) * NT * 128; }
+  static __host__ __device__ size_t q_bytes(int W) {
+    return QS ? 0 : static_cast<size_t>(W / 64) * NT * 128;
+  }
   static __host__ __device__ size_t bytes(int W, int stages) {
-    return 1024 + q_bytes(W) + static_cast<size_t>(stages) * kSlice +
+    return 1024 + q_bytes(W) + static_cast<size_t>(stages) * kStage +
            static_cast<size_t>(kTileC) * kLD * 4 + (2 * kTileC + 8) * 4 + (2 * stages + 7) * 8 +
            32;
   }
 };
 
-template <int NT>
+template <int NT, bool QS>
 __global__ void __launch_bounds__(192, 1)
 route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                 int64_t C, int R, int W, int T_tok, float inv_Hr,
                 const int32_t *__restrict__ chunk_doc, int n_docs, float *__restrict__ state,
                 int n_chunk_tiles, int n_tiles, int stages) {
-  using L = RouteTcLayout<NT>;
+  using L = RouteTcLayout<NT, QS>;
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "UMMA N");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -54,7 +64,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   const int KS = W / 64;
   uint8_t *Qs = smem;
   uint8_t *Ks = Qs + L::q_bytes(W);
-  float *Sb = reinterpret_cast<float *>(Ks + static_cast<size_t>(stages) * L::kSlice);
+  float *Sb = reinterpret_cast<float *>(Ks + static_cast<size_t>(stages) * L::kStage);
   int *docs = reinterpret_cast<int *>(Sb + L::kTileC * L::kLD);
   int *segs = docs + L::kTileC;  // kTileC + 1 run starts (+ padding)
   uint64_t *bars = reinterpret_cast<uint64_t *>(segs + L::kTileC + 8);
@@ -106,7 +116,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       int it = 0, qloads = 0, cur_rt = -1;
       for (int tile = blockIdx.x; tile < n_tiles && !*fail; tile += gridDim.x) {
         const int rt = tile / n_chunk_tiles, ct = tile % n_chunk_tiles;
-        if (rt != cur_rt) {
+        if (!QS && rt != cur_rt) {
           if (qloads > 0 && !wait(qempty, (qloads - 1) & 1)) break;
           mbar_arrive_expect_tx(qfull, static_cast<uint32_t>(KS * NT * 128));
           for (int s = 0; s < KS; ++s)
@@ -117,9 +127,12 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         for (int s = 0; s < KS; ++s) {
           const int st = it % stages;
           if (it >= stages && !wait(empty0 + 8 * st, ((it / stages) - 1) & 1)) break;
-          mbar_arrive_expect_tx(full0 + 8 * st, L::kSlice);
-          tma_load_2d_hint(ks_addr + st * L::kSlice, &tmK, 64 * s, ct * L::kTileC,
+          mbar_arrive_expect_tx(full0 + 8 * st, L::kStage);
+          tma_load_2d_hint(ks_addr + st * L::kStage, &tmK, 64 * s, ct * L::kTileC,
                            full0 + 8 * st, pol);
+          if (QS)
+            tma_load_2d(ks_addr + st * L::kStage + L::kSlice, &tmQ, 64 * s, rt * NT,
+                        full0 + 8 * st);
           ++it;
         }
       }
@@ -137,7 +150,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       bool issued = false;
       for (int tile = blockIdx.x; tile < n_tiles && !*fail; tile += gridDim.x, ++tl) {
         const int rt = tile / n_chunk_tiles;
-        if (rt != cur_rt) {
+        if (!QS && rt != cur_rt) {
           if (quses > 0) umma_commit(qempty);  // previous row tile's MMAs are all issued
           if (!wait(qfull, quses & 1)) break;
           ++quses;
@@ -152,8 +165,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
           const int st = it % stages;
           if (!wait(full0 + 8 * st, (it / stages) & 1)) { ok = false; break; }
           tc05_fence_after();
-          const uint32_t a0 = ks_addr + st * L::kSlice;
-          const uint32_t b0 = qs_addr + s * NT * 128;
+          const uint32_t a0 = ks_addr + st * L::kStage;
+          const uint32_t b0 = QS ? a0 + L::kSlice : qs_addr + s * NT * 128;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16(d_tmem, umma_desc_k_sw128(a0 + kk * 32), umma_desc_k_sw128(b0 + kk * 32),
@@ -203,12 +216,14 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       asm volatile("bar.sync 1, 128;" ::: "memory");
       // after a failed wait the results are void (the error word is set): skip the epilogue
       const bool go = !*fail;
-      if (go) epi_token_max(Sb, L::kLD, MC, NR, r0, T_tok, tid, 128);
+      if (go && T_tok > 1) epi_token_max(Sb, L::kLD, MC, NR, r0, T_tok, tid, 128);
       asm volatile("bar.sync 1, 128;" ::: "memory");
-      const int64_t b0 = r0 / T_tok;
-      const int QB = static_cast<int>((r0 + NR - 1) / T_tok - b0 + 1);
-      int q_lo, q_hi;
-      query_span(r0, NR, T_tok, b0, q_lo, q_hi);
+      // (32-bit: r0 + NR <= R, an int)
+      const int r0i = static_cast<int>(r0);
+      const int b0 = r0i / T_tok;
+      const int QB = (r0i + NR - 1) / T_tok - b0 + 1;
+      const int q_lo = (r0i + T_tok - 1) / T_tok - b0;  // queries with all T rows in the tile
+      const int q_hi = max(q_lo, (r0i + NR) / T_tok - b0);
       epi_doc_max(Sb, L::kLD, MC, QB, b0, docs, prev_doc, next_doc, q_lo, q_hi, n_docs, state,
                   segs, tid, 128, go);
       asm volatile("bar.sync 1, 128;" ::: "memory");
