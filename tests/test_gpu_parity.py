@@ -124,6 +124,37 @@ def test_document_encoded_alone_is_byte_identical(case):
         assert torch.equal(rm1, rmean[cho[d]:cho[d + 1]])
 
 
+@pytest.mark.parametrize("case", ["ragged_bf16", "tiny_f32"])
+def test_incremental_update_of_one_document_equals_full_encode(case):
+    """Replacing one document's tokens and re-encoding only that document gives exactly the rows
+    a full encode of the updated memory gives, and leaves every other document's rows untouched:
+    document-wise RoPE makes a document's pooled rows depend on its own tokens alone."""
+    w = _workload(case)
+    inp = memory_inputs(w, seed=102)
+    mem = _build(w, inp)
+    rk, ct, rmean = _encode(mem, inp)
+    off, cho = inp["off"], mem.doc_chunk_offsets
+    d = mem.n_docs // 3
+    t0, t1 = int(off[d]), int(off[d + 1])
+    gen = torch.Generator().manual_seed(7)
+    new = {}
+    for n in ("K", "V", "Kr"):
+        x = inp[n].clone()
+        x[t0:t1] = torch.randn(x[t0:t1].shape, generator=gen).to(x.dtype)
+        new[n] = x
+    before = (rk.clone(), ct.clone(), rmean.clone())
+    mem.encode(d, 1, new["K"][t0:t1].cuda(), new["V"][t0:t1].cuda(), new["Kr"][t0:t1].cuda(), rk,
+               ct, rmean)
+    torch.cuda.synchronize()
+    full = _encode(mem, dict(inp, **new))
+    keep = torch.ones(rk.shape[0], dtype=torch.bool, device="cuda")
+    keep[int(cho[d]):int(cho[d + 1])] = False
+    for got, ref, old in zip((rk, ct, rmean), full, before):
+        assert torch.equal(got, ref)
+        assert torch.equal(got[keep], old[keep])
+        assert not torch.equal(got[~keep], old[~keep])
+
+
 def _check_topk(ids, scores, state, ref_state, k, tol, eligible=None):
     """ids/scores from the GPU; ref_state from the oracle (fp64)."""
     ids, scores, state = ids.cpu().numpy(), scores.cpu().numpy(), state.cpu().numpy()

@@ -8,7 +8,7 @@
 //   append_kernel         rotate the new K rows, write K/V into the local cache
 //   attend_simt_kernel    fp32 path (CUDA cores, one warp per query head)
 //   attend_mma_kernel     bf16 path: per (query, kv head, token, context
-//                         split) CTA, 4 warps stream 16-row context blocks
+//                         split) CTA, 3 warps stream 16-row context blocks
 //                         (cp.async, double-buffered, XOR-swizzled smem) and
 //                         run S = Q K^T and O += P V on mma.sync with an
 //                         online softmax; the GQA group's heads are the M rows
@@ -207,7 +207,9 @@ attend_simt_kernel(const T *__restrict__ content, const int32_t *__restrict__ id
 }
 
 // ---------------------------------------------------------------- bf16 path
-constexpr int kAttWarps = 4;
+// Three warps per CTA: 3 x 2 stages x 2 x 16 x D x 2 B of ring (48 KB at D = 128) lets four
+// CTAs share an SM, so the 8 x 64 (query, kv head) CTAs of a decode batch run in one wave.
+constexpr int kAttWarps = 3;
 constexpr int kAttRows = 16;  // context rows per warp block
 
 template <int D>
@@ -229,9 +231,9 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return static_cast<uint32_t>(r * (D * 2) + ((c ^ (r & 7)) << 4));
 }
 
-// grid (B * H_kv, n_split, T), block 128.
+// grid (B * H_kv, n_split, T), block 32 * kAttWarps.
 template <int D, int G>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(32 * kAttWarps)
 attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__restrict__ ids,
                   int k, const int64_t *__restrict__ doc_chunk_off, int n_docs,
                   const int32_t *__restrict__ slots, int slot_chunks, int H_kv,

@@ -144,7 +144,7 @@ size_t elem_size(msa_dtype t) { return t == MSA_BF16 ? 2 : 4; }
 int topk_splits(int n_docs) { return (n_docs + msa::kTopkSlice - 1) / msa::kTopkSlice; }
 
 // Context splits of one attention launch: enough CTAs for about three per
-// SM (the kernel's residency); more splits only add per-CTA fixed cost and
+// SM (the kernel holds four); more splits only add per-CTA fixed cost and
 // combine traffic (measured on the 1M- and 100M-token decode workloads).
 int attend_splits(int B, int T, int H_kv, int64_t max_ctx) {
   const int64_t ctas = static_cast<int64_t>(B) * T * H_kv;
