@@ -4,7 +4,8 @@
 // id).  Each (score, id) pair is packed into one order-preserving 64-bit key,
 // so the top-k is a selection of the k largest keys -- exact and
 // deterministic.  Phase 1: one CTA per (query, 4096-document slice) selects
-// its slice's k largest keys; phase 2 merges the slices' candidates.
+// its slice's k largest keys; phase 2 merges the slices' candidates.  Both
+// filter first (block_select_topk_fast) and sort only the few survivors.
 #pragma once
 #include "common.cuh"
 
@@ -104,6 +105,83 @@ __device__ __forceinline__ void block_select_topk(const unsigned long long (&key
   __syncthreads();
 }
 
+// --- filtered selection ------------------------------------------------------
+// For k <= 32 most keys cannot be in the top k and need no sorting.  Each lane
+// takes the max of its keys; each warp sorts its 32 lane maxima (a 15-step
+// shuffle network) and its k-th largest t_w bounds the warp's own top k from
+// below: at least k of its keys are >= t_w (t_w = 1, i.e. every valid key,
+// when fewer than k lanes hold a key).  So the block holds at least k keys >=
+// T = max_w t_w and its top k are among them.  Those candidates (usually a few
+// more than k) are compacted into shared memory and ranked by counting (keys
+// are unique).  When they overflow kTopkCandCap (an adversarial layout of the
+// keys over the lanes) the block falls back to the sorting network above, so
+// the result is exact either way.
+constexpr int kTopkCandCap = 512;
+
+// descending bitonic sort of one key per lane across the warp
+__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long v, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, stride);
+      const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0);
+      v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+    }
+  return v;
+}
+
+// Same contract as block_select_topk.  Shared scratch: wt[kTopkWarps + 1] and
+// cbuf[kTopkCandCap] besides block_select_topk's.
+template <int KL>
+__device__ __forceinline__ void block_select_topk_fast(
+    const unsigned long long (&key)[kTopkPerThread], int k, unsigned long long *cand,
+    unsigned long long *sel, unsigned long long *wt, unsigned long long *cbuf) {
+  if (k > 32) {
+    block_select_topk<KL>(key, k, cand, sel);
+    return;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned long long m = 0ull;
+#pragma unroll
+  for (int j = 0; j < kTopkPerThread; ++j) m = key[j] > m ? key[j] : m;
+  m = warp_sort_desc(m, lane);
+  const unsigned long long tw = __shfl_sync(0xffffffffu, m, k - 1);
+  if (lane == 0) wt[warp] = tw ? tw : 1ull;
+  if (threadIdx.x == 0) wt[kTopkWarps] = 0ull;  // candidate count
+  __syncthreads();
+  unsigned long long T = 1ull;
+#pragma unroll
+  for (int w = 0; w < kTopkWarps; ++w) T = wt[w] > T ? wt[w] : T;
+  // compact the keys >= T (warp-aggregated slots)
+  unsigned int *count = reinterpret_cast<unsigned int *>(&wt[kTopkWarps]);
+#pragma unroll
+  for (int j = 0; j < kTopkPerThread; ++j) {
+    const bool in = key[j] >= T;
+    const unsigned bal = __ballot_sync(0xffffffffu, in);
+    if (bal == 0u) continue;
+    unsigned base = 0;
+    if (lane == 0) base = atomicAdd(count, static_cast<unsigned>(__popc(bal)));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const unsigned pos = base + __popc(bal & ((1u << lane) - 1u));
+    if (in && pos < kTopkCandCap) cbuf[pos] = key[j];
+  }
+  __syncthreads();
+  const unsigned n = *count;
+  if (n > kTopkCandCap) {  // uniform: every thread read the same count
+    block_select_topk<KL>(key, k, cand, sel);
+    return;
+  }
+  for (unsigned i = threadIdx.x; i < n; i += kTopkThreads) {
+    const unsigned long long x = cbuf[i];
+    int r = 0;
+    for (unsigned j2 = 0; j2 < n; ++j2) r += cbuf[j2] > x;
+    if (r < k) sel[r] = x;
+  }
+  for (int r = static_cast<int>(n) + threadIdx.x; r < k; r += kTopkThreads) sel[r] = 0ull;
+  __syncthreads();
+}
+
 __device__ __forceinline__ void write_topk(const unsigned long long *sel, int k, int32_t *ids,
                                            float *scores) {
   for (int r = threadIdx.x; r < k; r += kTopkThreads) {
@@ -122,6 +200,7 @@ topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__
                     int32_t *__restrict__ ids, float *__restrict__ scores) {
   __shared__ unsigned long long wc[kTopkWarps * KL];
   __shared__ unsigned long long sel[kMaxTopK];
+  __shared__ unsigned long long wt[kTopkWarps + 1], cbuf[kTopkCandCap];
   const int b = blockIdx.y, split = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(b) * n_docs;
@@ -133,7 +212,7 @@ topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__
     if (ok && exclude != nullptr) ok = exclude[row + d] == 0;
     key[j] = ok ? topk_key(state[row + d], d) : 0ull;
   }
-  block_select_topk<KL>(key, k, wc, sel);
+  block_select_topk_fast<KL>(key, k, wc, sel, wt, cbuf);
   if (n_split == 1) {
     write_topk(sel, k, ids + static_cast<int64_t>(b) * k, scores + static_cast<int64_t>(b) * k);
   } else {
@@ -149,6 +228,7 @@ topk_merge_kernel(const unsigned long long *__restrict__ cand, int n_cand, int k
                   int32_t *__restrict__ ids, float *__restrict__ scores) {
   __shared__ unsigned long long wc[kTopkWarps * KL];
   __shared__ unsigned long long sel[kMaxTopK];
+  __shared__ unsigned long long wt[kTopkWarps + 1], cbuf[kTopkCandCap];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned long long key[kTopkPerThread];
@@ -157,7 +237,7 @@ topk_merge_kernel(const unsigned long long *__restrict__ cand, int n_cand, int k
     const int i = warp * (32 * kTopkPerThread) + j * 32 + lane;
     key[j] = i < n_cand ? cand[static_cast<int64_t>(b) * n_cand + i] : 0ull;
   }
-  block_select_topk<KL>(key, k, wc, sel);
+  block_select_topk_fast<KL>(key, k, wc, sel, wt, cbuf);
   write_topk(sel, k, ids + static_cast<int64_t>(b) * k, scores + static_cast<int64_t>(b) * k);
 }
 
