@@ -257,6 +257,8 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
   const int b = blockIdx.x / H_kv, g = blockIdx.x % H_kv;
   const int split = blockIdx.y, i = blockIdx.z;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  griddep_wait();
+  griddep_launch();
 
   const int n_mem = build_chunk_table(ids + static_cast<int64_t>(b) * k, k, doc_chunk_off, n_docs,
                                       slots ? slots + static_cast<int64_t>(b) * k : nullptr,
@@ -516,6 +518,8 @@ __global__ void attend_combine_kernel(const float *__restrict__ part_o,
                                       const float *__restrict__ part_ml, int n_split, int D,
                                       __nv_bfloat16 *__restrict__ O, int32_t *__restrict__ cache_len,
                                       int rows_per_query, int T_tok, int cap) {
+  griddep_wait();
+  griddep_launch();
   const int64_t orow = blockIdx.x;
   if (threadIdx.x == 0 && orow % rows_per_query == 0) {
     int32_t *cl = cache_len + orow / rows_per_query;
@@ -537,6 +541,8 @@ __global__ void attend_combine_kernel(const float *__restrict__ part_o,
 }
 
 __global__ void advance_kernel(int32_t *__restrict__ cache_len, int B, int T_tok, int cap) {
+  griddep_wait();
+  griddep_launch();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) cache_len[b] = min(cache_len[b] + T_tok, cap);
 }

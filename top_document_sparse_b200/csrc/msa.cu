@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
+#include <utility>
 
 #include "attend.cuh"
 #include "common.cuh"
@@ -58,6 +59,27 @@ std::atomic<uint64_t> g_launches{0};
     if (e_ != cudaSuccess) return cuda_fail(e_, what);  \
     g_launches.fetch_add(1, std::memory_order_relaxed); \
   } while (0)
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on the stream drains (it calls griddep_wait() before
+// its first global memory access), which hides the launch and the kernel's
+// setup behind the previous kernel's tail.  Used for the per-token decode
+// path, where a step is a chain of short dependent kernels.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Device address of the static attention scratch on the current device, looked
 // up once per device (cudaGetSymbolAddress with that device current).
@@ -218,9 +240,9 @@ msa_status launch_route_tc(const msa_memory *mem, const void *keys, const void *
   const int64_t n_tiles = static_cast<int64_t>(n_ct) * n_rt;
   if (n_tiles > INT32_MAX) return fail(MSA_ERR_UNSUPPORTED, "too many route tiles");
   const int grid = static_cast<int>(std::min<int64_t>(n_tiles, num_sms()));
-  kern<<<grid, 192, smem, st>>>(tmK, tmQ, mem->n_chunks, R, W, T, 1.0f / mem->H_r,
-                                mem->d_chunk_doc, mem->n_docs, state, n_ct,
-                                static_cast<int>(n_tiles), stages);
+  MSA_CUDA(launch_pdl(kern, dim3(grid), dim3(192), smem, st, tmK, tmQ, mem->n_chunks, R, W, T,
+                      1.0f / mem->H_r, mem->d_chunk_doc, mem->n_docs, state, n_ct,
+                      static_cast<int>(n_tiles), stages));
   MSA_LAUNCHED("route_tc_kernel");
   return MSA_OK;
 }
@@ -229,11 +251,12 @@ template <int KL>
 msa_status launch_topk(const msa_memory *mem, const float *state, const uint8_t *exclude, int B,
                        int k, int n_split, unsigned long long *cand, int32_t *ids, float *scores,
                        cudaStream_t st) {
-  msa::topk_partial_kernel<KL><<<dim3(n_split, B), msa::kTopkThreads, 0, st>>>(
-      state, exclude, mem->n_docs, k, n_split, cand, ids, scores);
+  MSA_CUDA(launch_pdl(msa::topk_partial_kernel<KL>, dim3(n_split, B), dim3(msa::kTopkThreads), 0,
+                      st, state, exclude, mem->n_docs, k, n_split, cand, ids, scores));
   MSA_LAUNCHED("topk_partial_kernel");
   if (n_split > 1) {
-    msa::topk_merge_kernel<KL><<<B, msa::kTopkThreads, 0, st>>>(cand, n_split * k, k, ids, scores);
+    MSA_CUDA(launch_pdl(msa::topk_merge_kernel<KL>, dim3(B), dim3(msa::kTopkThreads), 0, st,
+                        static_cast<const unsigned long long *>(cand), n_split * k, k, ids, scores));
     MSA_LAUNCHED("topk_merge_kernel");
   }
   return MSA_OK;
@@ -267,8 +290,8 @@ msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, i
     const int thr = round32(W / 4);
     if (mem->dtype == MSA_BF16) {
       auto *qh = reinterpret_cast<__nv_bfloat16 *>(wsb + plan.qhat);
-      msa::qnorm_kernel<__nv_bfloat16><<<R, thr, 0, st>>>(
-          static_cast<const __nv_bfloat16 *>(Qr), W, mem->d_r, T, q_pitch, qh);
+      MSA_CUDA(launch_pdl(msa::qnorm_kernel<__nv_bfloat16>, dim3(R), dim3(thr), 0, st,
+                          static_cast<const __nv_bfloat16 *>(Qr), W, mem->d_r, T, q_pitch, qh));
       MSA_LAUNCHED("qnorm_kernel");
       msa_status s;
       if (R <= 16)
@@ -314,23 +337,27 @@ msa_status launch_attend_mma(const msa_memory *mem, const void *content, const i
   const float scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)) * 1.4426950408889634);
   const int fuse_append = T == 1 ? 1 : 0;
   dim3 grid(static_cast<unsigned>(B * mem->H_kv), plan.n_split, T);
-  kern<<<grid, 32 * msa::kAttWarps, smem, st>>>(
-      static_cast<const __nv_bfloat16 *>(content), ids, k, mem->d_doc_chunk_off, mem->n_docs, slots,
-      slot_chunks, mem->H_kv, static_cast<const __nv_bfloat16 *>(Q), T,
-      static_cast<__nv_bfloat16 *>(Kc), static_cast<__nv_bfloat16 *>(Vc),
-      static_cast<const __nv_bfloat16 *>(K_new), static_cast<const __nv_bfloat16 *>(V_new),
-      cache_len, cap, pos_offset, mem->d_rope, scale_log2, plan.n_split, plan.table_cap,
-      fuse_append, static_cast<__nv_bfloat16 *>(O), part_o, part_ml);
+  MSA_CUDA(launch_pdl(
+      kern, grid, dim3(32 * msa::kAttWarps), smem, st,
+      static_cast<const __nv_bfloat16 *>(content), ids, k,
+      static_cast<const int64_t *>(mem->d_doc_chunk_off), mem->n_docs, slots, slot_chunks,
+      mem->H_kv, static_cast<const __nv_bfloat16 *>(Q), T, static_cast<__nv_bfloat16 *>(Kc),
+      static_cast<__nv_bfloat16 *>(Vc), static_cast<const __nv_bfloat16 *>(K_new),
+      static_cast<const __nv_bfloat16 *>(V_new), static_cast<const int32_t *>(cache_len), cap,
+      pos_offset, static_cast<const float2 *>(mem->d_rope), scale_log2, plan.n_split,
+      plan.table_cap, fuse_append, static_cast<__nv_bfloat16 *>(O), part_o, part_ml));
   MSA_LAUNCHED("attend_mma_kernel");
   if (plan.n_split > 1) {
     // merge the splits and advance cache_len (every attention CTA has read it)
-    msa::attend_combine_kernel<<<static_cast<unsigned>(static_cast<int64_t>(B) * T * mem->H_kv * G),
-                                 D, 0, st>>>(part_o, part_ml, plan.n_split, D,
-                                             static_cast<__nv_bfloat16 *>(O), cache_len,
-                                             T * mem->H_kv * G, T, cap);
+    MSA_CUDA(launch_pdl(msa::attend_combine_kernel,
+                        dim3(static_cast<unsigned>(static_cast<int64_t>(B) * T * mem->H_kv * G)),
+                        dim3(D), 0, st, static_cast<const float *>(part_o),
+                        static_cast<const float *>(part_ml), plan.n_split, D,
+                        static_cast<__nv_bfloat16 *>(O), cache_len, T * mem->H_kv * G, T, cap));
     MSA_LAUNCHED("attend_combine_kernel");
   } else {
-    msa::advance_kernel<<<(B + 255) / 256, 256, 0, st>>>(cache_len, B, T, cap);
+    MSA_CUDA(launch_pdl(msa::advance_kernel, dim3((B + 255) / 256), dim3(256), 0, st, cache_len, B,
+                        T, cap));
     MSA_LAUNCHED("advance_kernel");
   }
   return MSA_OK;

@@ -123,6 +123,22 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the kernel before it on the stream drains;
+// griddep_wait() blocks until that kernel has completed and its memory is
+// visible.  Every kernel launched that way calls it before its first global
+// memory access (it is a no-op for an ordinary launch).
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Let the next kernel on the stream be scheduled now (it still waits for this
+// one's completion in its own griddep_wait()); called right after
+// griddep_wait(), so at most one kernel ahead is resident early.
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);

@@ -20,6 +20,8 @@ namespace msa {
 template <typename T>
 __global__ void qnorm_kernel(const T *__restrict__ Qr, int W, int d_r, int T_tok, int pitch,
                              T *__restrict__ out) {
+  griddep_wait();
+  griddep_launch();
   const int64_t r = blockIdx.x;
   const int64_t src_row = (r / T_tok) * pitch + r % T_tok;
   const int e0 = threadIdx.x * 4;

@@ -98,6 +98,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   __syncthreads();
   tc05_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // setup above overlaps the previous kernel's drain
+  griddep_launch();
 
   auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
     if (*fail) return false;

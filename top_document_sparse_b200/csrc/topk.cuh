@@ -8,6 +8,7 @@
 // filter first (block_select_topk_fast) and sort only the few survivors.
 #pragma once
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace msa {
 
@@ -204,6 +205,8 @@ topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__
   const int b = blockIdx.y, split = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(b) * n_docs;
+  griddep_wait();
+  griddep_launch();
   unsigned long long key[kTopkPerThread];
 #pragma unroll
   for (int j = 0; j < kTopkPerThread; ++j) {
@@ -231,6 +234,8 @@ topk_merge_kernel(const unsigned long long *__restrict__ cand, int n_cand, int k
   __shared__ unsigned long long wt[kTopkWarps + 1], cbuf[kTopkCandCap];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_wait();
+  griddep_launch();
   unsigned long long key[kTopkPerThread];
 #pragma unroll
   for (int j = 0; j < kTopkPerThread; ++j) {
