@@ -324,8 +324,8 @@ MSA_API msa_status msa_interleave(const msa_memory *mem, const void *router_keys
  *   flags        : MSA_FETCH_COLD forgets every resident document at each
  *                  fetch (every selected document crosses the host link)
  * The fetcher allocates small host-side tables, two events, pinned host
- * staging for max_batch * max_k ids and slots, and a device array of the same
- * size; it does not own content_host or slot_cache.
+ * staging for max_batch * max_k ids, slots and copy-list entries, and device
+ * arrays of the same sizes; it does not own content_host or slot_cache.
  */
 typedef struct msa_fetcher msa_fetcher;
 #define MSA_FETCH_COLD 0x1u
@@ -343,10 +343,12 @@ MSA_API msa_status msa_fetcher_stats(const msa_fetcher *f, int64_t *hits, int64_
  * Make the documents ids[batch][k] (device) resident in the slot cache.
  * Reads the ids back to the host (synchronising `stream` up to that copy),
  * keeps resident documents, chooses victim slots (a clock over the slots not
- * used by this call) for the others and copies each missing document (one
- * cudaMemcpyAsync of its contiguous chunk rows) on `fetch_stream`, uploads
- * the slot of every (query, rank), and makes `stream` wait for
- * `fetch_stream`.  Ids outside [0, n_docs) get slot 0 and are skipped by the
+ * used by this call) for the others and, on `fetch_stream`, uploads the slot
+ * of every (query, rank) and copies every missing document's contiguous chunk
+ * rows over the host link: one gather kernel reading content_host through its
+ * device mapping (one CTA per document), or one cudaMemcpyAsync per document
+ * when content_host is not mapped into the device address space.  Then makes
+ * `stream` wait for `fetch_stream`.  Ids outside [0, n_docs) get slot 0 and are skipped by the
  * attention (device error word).  fetch_stream may equal stream.
  */
 MSA_API msa_status msa_fetch(msa_fetcher *f, const int32_t *ids, int32_t batch, int32_t k,

@@ -779,11 +779,19 @@ msa_status msa_fetcher_create(const msa_memory *mem, const void *content_host, v
       cudaHostAlloc(reinterpret_cast<void **>(&f->h_slots), n * 4, cudaHostAllocDefault) != cudaSuccess ||
       cudaMalloc(reinterpret_cast<void **>(&f->d_slots), n * 4) != cudaSuccess ||
       cudaEventCreateWithFlags(&f->ev_ids, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&f->ev_fetch, cudaEventDisableTiming) != cudaSuccess) {
+      cudaEventCreateWithFlags(&f->ev_fetch, cudaEventDisableTiming) != cudaSuccess ||
+      cudaHostAlloc(reinterpret_cast<void **>(&f->h_list), n * 3 * 8, cudaHostAllocDefault) != cudaSuccess ||
+      cudaMalloc(reinterpret_cast<void **>(&f->d_list), n * 3 * 8) != cudaSuccess) {
     cudaGetLastError();
     msa_fetcher_destroy(f);
     return fail(MSA_ERR_OUT_OF_MEMORY, "could not allocate the fetcher's staging buffers");
   }
+  // the gather kernel reads the content through its device mapping when it has one
+  void *dev = nullptr;
+  if (cudaHostGetDevicePointer(&dev, const_cast<void *>(content_host), 0) == cudaSuccess && dev)
+    f->content_dev = static_cast<const uint8_t *>(dev);
+  else
+    cudaGetLastError();
   *out = f;
   return MSA_OK;
 }
@@ -793,6 +801,8 @@ msa_status msa_fetcher_destroy(msa_fetcher *f) {
   if (f->h_ids) cudaFreeHost(f->h_ids);
   if (f->h_slots) cudaFreeHost(f->h_slots);
   if (f->d_slots) cudaFree(f->d_slots);
+  if (f->h_list) cudaFreeHost(f->h_list);
+  if (f->d_list) cudaFree(f->d_list);
   if (f->ev_ids) cudaEventDestroy(f->ev_ids);
   if (f->ev_fetch) cudaEventDestroy(f->ev_fetch);
   delete f;
@@ -829,6 +839,7 @@ msa_status msa_fetch(msa_fetcher *f, const int32_t *ids, int32_t batch, int32_t 
     }
   }
   const msa_memory *mem = f->mem;
+  int n_miss = 0;
   // resident documents keep their slots
   for (int i = 0; i < n; ++i) {
     const int d = f->h_ids[i];
@@ -859,14 +870,27 @@ msa_status msa_fetch(msa_fetcher *f, const int32_t *ids, int32_t batch, int32_t 
     f->h_slots[i] = s;
     const int64_t c0 = mem->doc_chunk_off[d], c1 = mem->doc_chunk_off[d + 1];
     const size_t nb = static_cast<size_t>(c1 - c0) * f->row_bytes;
-    MSA_CUDA(cudaMemcpyAsync(f->slot_cache + static_cast<size_t>(s) * f->slot_bytes,
-                             f->content_host + static_cast<size_t>(c0) * f->row_bytes, nb,
-                             cudaMemcpyHostToDevice, fst));
+    if (f->content_dev) {
+      f->h_list[3 * n_miss] = static_cast<int64_t>(c0) * static_cast<int64_t>(f->row_bytes);
+      f->h_list[3 * n_miss + 1] = static_cast<int64_t>(nb);
+      f->h_list[3 * n_miss + 2] = static_cast<int64_t>(s) * static_cast<int64_t>(f->slot_bytes);
+    } else {
+      MSA_CUDA(cudaMemcpyAsync(f->slot_cache + static_cast<size_t>(s) * f->slot_bytes,
+                               f->content_host + static_cast<size_t>(c0) * f->row_bytes, nb,
+                               cudaMemcpyHostToDevice, fst));
+    }
+    ++n_miss;
     ++f->misses;
     ++f->copies;
     f->bytes += static_cast<int64_t>(nb);
   }
   MSA_CUDA(cudaMemcpyAsync(f->d_slots, f->h_slots, n * sizeof(int32_t), cudaMemcpyHostToDevice, fst));
+  if (f->content_dev && n_miss > 0) {
+    MSA_CUDA(cudaMemcpyAsync(f->d_list, f->h_list, static_cast<size_t>(n_miss) * 3 * 8,
+                             cudaMemcpyHostToDevice, fst));
+    msa::fetch_gather_kernel<<<n_miss, 256, 0, fst>>>(f->content_dev, f->slot_cache, f->d_list);
+    MSA_LAUNCHED("fetch_gather_kernel");
+  }
   if (fst != st) {
     MSA_CUDA(cudaEventRecord(f->ev_fetch, fst));
     MSA_CUDA(cudaStreamWaitEvent(st, f->ev_fetch, 0));
