@@ -10,8 +10,9 @@
 //   attend_mma_kernel     bf16 path: per (query, kv head, token, context
 //                         split) CTA, 3 warps stream 16-row context blocks
 //                         (cp.async, double-buffered, XOR-swizzled smem) and
-//                         run S = Q K^T and O += P V on mma.sync with an
-//                         online softmax; the GQA group's heads are the M rows
+//                         run S^T = K Q^T and O^T += V^T P^T on mma.sync with
+//                         an online softmax (context rows / head dim on M, the
+//                         GQA group's heads on N)
 //   attend_combine_kernel merge context splits (log-sum-exp) and advance
 //                         cache_len
 // For a one-token call (decode) the attention kernel appends the new row
@@ -350,24 +351,35 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
   }
   __syncthreads();
 
-  // A fragments of Q for every k-step
-  uint32_t qa[D / 16][4];
+  // Transposed tile: S^T = K Q^T (M = 16 context rows, N = 8 heads per n tile,
+  // K = D) and O^T += V^T P^T (M = D, N = heads, K = 16 context rows), P^T
+  // reaching the B operand through movmatrix, so no MMA row is spent on the
+  // GQA group's few heads.  A thread's accumulators hold heads
+  // nt * 8 + (lane & 3) * 2 + {0, 1} and rows d = dm * 16 + lane / 4 (+ 8);
+  // the online softmax state of a head is uniform over the 8 lane groups.
+  constexpr int NT = (G + 7) / 8;  // n8 tiles of heads
+  uint32_t qb[NT][D / 16][2];      // B fragments of Q^T (query rows >= G are zero)
   {
     const uint32_t qbase = smem_u32(qsm);
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const int r = lane & 15, c = 2 * kk + (lane >> 4);
-      ldsm_x4(qbase + swz<D>(r, c), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
-    }
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int kp = 0; kp < D / 32; ++kp)
+        ldsm_x4(qbase + swz<D>(nt * 8 + (lane & 7), 4 * kp + (lane >> 3)), qb[nt][2 * kp][0],
+                qb[nt][2 * kp][1], qb[nt][2 * kp + 1][0], qb[nt][2 * kp + 1][1]);
   }
 
-  float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 domain) of rows g8 and g8+8
-  float l0 = 0.0f, l1 = 0.0f;
-  float acc[D / 8][4];
+  float mh[NT][2], lh[NT][2];  // running max (log2 units) and partial sum per head
+  float acc[NT][D / 16][4];
 #pragma unroll
-  for (int n = 0; n < D / 8; ++n)
+  for (int nt = 0; nt < NT; ++nt) {
+    mh[nt][0] = mh[nt][1] = -INFINITY;
+    lh[nt][0] = lh[nt][1] = 0.0f;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[n][e] = 0.0f;
+    for (int dm = 0; dm < D / 16; ++dm)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nt][dm][e] = 0.0f;
+  }
 
   for (int bi = warp; bi < nblk; bi += kAttWarps) {
     const int x = x0 + bi * kAttRows;
@@ -381,107 +393,90 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
     const uint32_t kb = smem_u32(wbuf + s * 2 * Sm::kBlockBytes);
     const uint32_t vb = kb + Sm::kBlockBytes;
 
-    // S = Q K^T over 16 context rows (two n8 tiles)
-    float sc[2][4];
+    // S^T = K Q^T over the block's 16 context rows
+    float sc[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sc[nt][e] = 0.0f;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      const int r = (lane & 7) + ((lane >> 4) << 3), c = 2 * kk + ((lane >> 3) & 1);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(kb + swz<D>(r, c), b0, b1, b2, b3);
-      mma_bf16_16816(sc[0], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
-      mma_bf16_16816(sc[1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(kb + swz<D>(lane & 15, 2 * kk + (lane >> 4)), a0, a1, a2, a3);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        mma_bf16_16816(sc[nt], a0, a1, a2, a3, qb[nt][kk][0], qb[nt][kk][1]);
     }
-    // scale to log2 units, mask rows past the split end
-    float bm0 = -INFINITY, bm1 = -INFINITY;
+    // online softmax per head over context rows x + lane/4 (c0, c1) and + 8 (c2, c3),
+    // in log2 units; rows past the split end are masked
+    const bool v0 = x + (lane >> 2) < x1, v1 = x + (lane >> 2) + 8 < x1;
+    uint32_t pb[NT][2];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < NT; ++nt) {
+      float al[2];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int col = x + nt * 8 + (lane & 3) * 2 + e;
-        const bool ok = col < x1;
-        sc[nt][e] = ok ? sc[nt][e] * scale_log2 : -INFINITY;
-        sc[nt][2 + e] = ok ? sc[nt][2 + e] * scale_log2 : -INFINITY;
-        bm0 = fmaxf(bm0, sc[nt][e]);
-        bm1 = fmaxf(bm1, sc[nt][2 + e]);
+      for (int h = 0; h < 2; ++h) {
+        const float s0 = v0 ? sc[nt][h] * scale_log2 : -INFINITY;
+        const float s1 = v1 ? sc[nt][2 + h] * scale_log2 : -INFINITY;
+        float bm = fmaxf(s0, s1);
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+        const float mn = fmaxf(mh[nt][h], bm);  // finite: every block has a context row
+        al[h] = exp2f(mh[nt][h] - mn);
+        mh[nt][h] = mn;
+        sc[nt][h] = exp2f(s0 - mn);
+        sc[nt][2 + h] = exp2f(s1 - mn);
+        lh[nt][h] = lh[nt][h] * al[h] + sc[nt][h] + sc[nt][2 + h];
       }
 #pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-      bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, o));
-      bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, o));
-    }
-    const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
-    const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
-    const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
-    const float al0 = exp2f(m0 - base0), al1 = exp2f(m1 - base1);
-    m0 = mn0;
-    m1 = mn1;
-    float ps0 = 0.0f, ps1 = 0.0f;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        sc[nt][e] = exp2f(sc[nt][e] - base0);
-        sc[nt][2 + e] = exp2f(sc[nt][2 + e] - base1);
-        ps0 += sc[nt][e];
-        ps1 += sc[nt][2 + e];
+      for (int dm = 0; dm < D / 16; ++dm) {
+        acc[nt][dm][0] *= al[0];
+        acc[nt][dm][1] *= al[1];
+        acc[nt][dm][2] *= al[0];
+        acc[nt][dm][3] *= al[1];
       }
-    l0 = l0 * al0 + ps0;
-    l1 = l1 * al1 + ps1;
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      acc[n][0] *= al0;
-      acc[n][1] *= al0;
-      acc[n][2] *= al1;
-      acc[n][3] *= al1;
+      // P^T as the B operand: transpose the two 8x8 bf16 quadrants in registers
+      pb[nt][0] = movmatrix_trans(pack_bf16x2(sc[nt][0], sc[nt][1]));
+      pb[nt][1] = movmatrix_trans(pack_bf16x2(sc[nt][2], sc[nt][3]));
     }
-    // O += P V
-    const uint32_t pa0 = pack_bf16x2(sc[0][0], sc[0][1]);
-    const uint32_t pa1 = pack_bf16x2(sc[0][2], sc[0][3]);
-    const uint32_t pa2 = pack_bf16x2(sc[1][0], sc[1][1]);
-    const uint32_t pa3 = pack_bf16x2(sc[1][2], sc[1][3]);
+    // O^T += V^T P^T
 #pragma unroll
-    for (int dp = 0; dp < D / 16; ++dp) {
-      const int r = (lane & 7) + (((lane >> 3) & 1) << 3), c = 2 * dp + (lane >> 4);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_trans(vb + swz<D>(r, c), b0, b1, b2, b3);
-      mma_bf16_16816(acc[2 * dp], pa0, pa1, pa2, pa3, b0, b1);
-      mma_bf16_16816(acc[2 * dp + 1], pa0, pa1, pa2, pa3, b2, b3);
+    for (int dm = 0; dm < D / 16; ++dm) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_trans(vb + swz<D>((lane & 7) + ((lane >> 4) << 3), 2 * dm + ((lane >> 3) & 1)), a0,
+                    a1, a2, a3);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        mma_bf16_16816(acc[nt][dm], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
     }
     __syncwarp();
     s ^= 1;
   }
 
-  // per-row totals across the 4 lanes of a row group
-#pragma unroll
-  for (int o = 1; o <= 2; o <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-  }
+  // per-head totals over the 8 lane groups; the warps merge through shared memory
   __syncthreads();  // every warp is done with the ring: reuse it for the merge
   float *mo = reinterpret_cast<float *>(ring);  // [warp][16][D + 2]: D outputs, m, l
-  {
-    const int r0 = lane >> 2;
-    float *row0 = mo + (warp * 16 + r0) * (D + 2);
-    float *row1 = mo + (warp * 16 + r0 + 8) * (D + 2);
 #pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      const int col = n * 8 + (lane & 3) * 2;
-      row0[col] = acc[n][0];
-      row0[col + 1] = acc[n][1];
-      row1[col] = acc[n][2];
-      row1[col + 1] = acc[n][3];
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float L = lh[nt][h];
+      L += __shfl_xor_sync(0xffffffffu, L, 4);
+      L += __shfl_xor_sync(0xffffffffu, L, 8);
+      L += __shfl_xor_sync(0xffffffffu, L, 16);
+      const int head = nt * 8 + (lane & 3) * 2 + h;
+      float *row = mo + (warp * 16 + head) * (D + 2);
+#pragma unroll
+      for (int dm = 0; dm < D / 16; ++dm) {
+        row[dm * 16 + (lane >> 2)] = acc[nt][dm][h];
+        row[dm * 16 + (lane >> 2) + 8] = acc[nt][dm][2 + h];
+      }
+      if (lane < 4) {
+        row[D] = mh[nt][h];
+        row[D + 1] = L;
+      }
     }
-    if ((lane & 3) == 0) {
-      row0[D] = m0;
-      row0[D + 1] = l0;
-      row1[D] = m1;
-      row1[D + 1] = l1;
-    }
-  }
   __syncthreads();
   for (int p = threadIdx.x; p < G * D; p += blockDim.x) {
     const int r = p / D, e = p % D;
