@@ -243,8 +243,8 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
                   const __nv_bfloat16 *__restrict__ K_new, const __nv_bfloat16 *__restrict__ V_new,
                   const int32_t *__restrict__ cache_len, int cap, int pos_offset,
                   const float2 *__restrict__ rope, float scale_log2, int n_split, int table_cap,
-                  int fuse_append, __nv_bfloat16 *__restrict__ O, float *__restrict__ part_o,
-                  float *__restrict__ part_ml) {
+                  int fuse_append, int early, __nv_bfloat16 *__restrict__ O,
+                  float *__restrict__ part_o, float *__restrict__ part_ml) {
   constexpr int CPR = D / 8;  // 16-byte chunks per row
   using Sm = AttSmem<D>;
   extern __shared__ __align__(128) uint8_t sm[];
@@ -258,44 +258,46 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
   const int b = blockIdx.x / H_kv, g = blockIdx.x % H_kv;
   const int split = blockIdx.y, i = blockIdx.z;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  griddep_wait();
-  griddep_launch();
-
-  const int n_mem = build_chunk_table(ids + static_cast<int64_t>(b) * k, k, doc_chunk_off, n_docs,
-                                      slots ? slots + static_cast<int64_t>(b) * k : nullptr,
-                                      slot_chunks, table, pre, base, table_cap);
-  const int j = cache_len[b] + i;
-  const bool overflow = j >= cap || j < 0;
-  const int n_ctx = overflow ? 0 : n_mem + j + 1;
-  int per = (n_ctx + n_split - 1) / n_split;
-  per = (per + kAttRows - 1) / kAttRows * kAttRows;
-  const int x0 = split * per;
-  const int x1 = min(n_ctx, x0 + per);
   const int64_t kv = static_cast<int64_t>(H_kv) * D;
-  if (fuse_append) {
-    // one-token call: the CTA whose range holds the new row (context row
-    // n_mem + j) rotates K_new at pos_offset + j and writes K and V to the
-    // cache before any of its copies can read that row
-    if (overflow) {
-      if (threadIdx.x == 0 && g == 0 && split == 0) raise_device_error(MSA_DEVERR_CACHE_OVERFLOW);
-    } else if (x0 <= n_mem + j && n_mem + j < x1) {
-      const int half = D / 2;
-      const int64_t src = static_cast<int64_t>(b) * kv + g * D;
-      const int64_t dst = (static_cast<int64_t>(b) * cap + j) * kv + g * D;
-      const float2 *cs = rope + static_cast<int64_t>(pos_offset + j) * half;
-      for (int e = threadIdx.x; e < half; e += blockDim.x) {
-        const float a = __bfloat162float(K_new[src + e]);
-        const float c = __bfloat162float(K_new[src + e + half]);
-        const float2 t = cs[e];
-        K_cache[dst + e] = __float2bfloat16_rn(a * t.x - c * t.y);
-        K_cache[dst + e + half] = __float2bfloat16_rn(c * t.x + a * t.y);
-        V_cache[dst + e] = V_new[src + e];
-        V_cache[dst + e + half] = V_new[src + e + half];
-      }
-      __threadfence();  // the row is read back below through cp.async (L2)
-      __syncthreads();
-    }
+  const int half = D / 2;
+  // Context order: [local rows 0..j (causal) | memory rows in rank order]; the
+  // softmax does not depend on it.  The local part needs only cache_len, Q,
+  // the new token and the local cache, not the retrieved ids: with `early`
+  // (the caller guarantees that the kernel before this one on the stream
+  // writes none of those) and one split, the CTA starts on it before waiting
+  // for the previous kernel, reading them through L2.
+  const bool early_ok = early && n_split == 1;
+  if (!early_ok) {
+    griddep_wait();
+    griddep_launch();
   }
+  const int j = (early_ok ? __ldcg(cache_len + b) : cache_len[b]) + i;
+  const bool overflow = j >= cap || j < 0;
+  const int n_loc = overflow ? 0 : j + 1;
+  int n_mem = 0, x0 = 0, x1 = n_loc;  // until the table is built, only local rows are issued
+
+  // one-token call: the CTA whose range holds the new row (local row j)
+  // rotates K_new at pos_offset + j and writes K and V to the cache before any
+  // of its copies can read that row
+  auto append_new_row = [&]() {
+    const int64_t src = static_cast<int64_t>(b) * kv + g * D;
+    const int64_t dst = (static_cast<int64_t>(b) * cap + j) * kv + g * D;
+    const float2 *cs = rope + static_cast<int64_t>(pos_offset + j) * half;
+    for (int e = threadIdx.x; e < half; e += blockDim.x) {
+      const float a = __bfloat162float(__ldcg(K_new + src + e));
+      const float c = __bfloat162float(__ldcg(K_new + src + e + half));
+      const float2 t = cs[e];
+      K_cache[dst + e] = __float2bfloat16_rn(a * t.x - c * t.y);
+      K_cache[dst + e + half] = __float2bfloat16_rn(c * t.x + a * t.y);
+      V_cache[dst + e] = __ldcg(V_new + src + e);
+      V_cache[dst + e + half] = __ldcg(V_new + src + e + half);
+    }
+    __threadfence();  // the row is read back through cp.async (L2)
+    __syncthreads();
+  };
+  if (fuse_append && overflow && threadIdx.x == 0 && g == 0 && split == 0)
+    raise_device_error(MSA_DEVERR_CACHE_OVERFLOW);
+  if (early_ok && fuse_append && !overflow) append_new_row();  // one split holds every row
 
   uint8_t *wbuf = ring + warp * Sm::kWarpBytes;
   // issue the loads of the block starting at context row x into stage s
@@ -310,13 +312,13 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
       const __nv_bfloat16 *ks = K_cache, *vs = V_cache;
       bool ok = xr < x1;
       if (ok) {
-        if (xr < n_mem) {
-          ks = content + static_cast<int64_t>(table[xr]) * 2 * kv + g * D;
-          vs = ks + kv;
-        } else {
-          const int64_t row = (static_cast<int64_t>(b) * cap + (xr - n_mem)) * kv + g * D;
+        if (xr < n_loc) {
+          const int64_t row = (static_cast<int64_t>(b) * cap + xr) * kv + g * D;
           ks = K_cache + row;
           vs = V_cache + row;
+        } else {
+          ks = content + static_cast<int64_t>(table[xr - n_loc]) * 2 * kv + g * D;
+          vs = ks + kv;
         }
       }
       cp_async_16(smem_u32(kb + swz<D>(r, c)), ks + c * 8, ok);
@@ -324,22 +326,22 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
     }
     cp_async_commit();
   };
-
-  // the first context block is in flight while the query is rotated
-  const int nblk = (x1 > x0) ? (x1 - x0 + kAttRows - 1) / kAttRows : 0;
-  int s = 0;
-  if (warp < nblk) issue(x0 + warp * kAttRows, 0);
+  // early: the first block of every warp is in flight before the wait if it is all local
+  bool issued = false;
+  if (early_ok && (warp + 1) * kAttRows <= n_loc) {
+    issue(warp * kAttRows, 0);
+    issued = true;
+  }
   // rotated query rows of the group -> qsm [16][D] (rows >= G are zero)
   {
-    const int half = D / 2;
     const __nv_bfloat16 *qb = Q + ((static_cast<int64_t>(b) * T_tok + i) * H_q + g * G) * D;
     const float2 *cs = rope + static_cast<int64_t>(pos_offset + (overflow ? 0 : j)) * half;
     for (int p = threadIdx.x; p < 16 * half; p += blockDim.x) {
       const int r = p / half, e = p % half;
       float lo = 0.0f, hi = 0.0f;
       if (r < G) {
-        const float a = __bfloat162float(qb[r * D + e]);
-        const float c = __bfloat162float(qb[r * D + e + half]);
+        const float a = __bfloat162float(__ldcg(qb + r * D + e));
+        const float c = __bfloat162float(__ldcg(qb + r * D + e + half));
         const float2 t = cs[e];
         lo = a * t.x - c * t.y;
         hi = c * t.x + a * t.y;
@@ -349,6 +351,23 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
       *reinterpret_cast<__nv_bfloat16 *>(qsm + swz<D>(r, (e + half) / 8) + (e % 8) * 2) = bhi;
     }
   }
+  if (early_ok) {
+    griddep_wait();
+    griddep_launch();
+  }
+  n_mem = build_chunk_table(ids + static_cast<int64_t>(b) * k, k, doc_chunk_off, n_docs,
+                            slots ? slots + static_cast<int64_t>(b) * k : nullptr, slot_chunks,
+                            table, pre, base, table_cap);
+  const int n_ctx = overflow ? 0 : n_loc + n_mem;
+  int per = (n_ctx + n_split - 1) / n_split;
+  per = (per + kAttRows - 1) / kAttRows * kAttRows;
+  x0 = split * per;
+  x1 = min(n_ctx, x0 + per);
+  if (!early_ok && fuse_append && !overflow && x0 <= j && j < x1) append_new_row();
+
+  const int nblk = (x1 > x0) ? (x1 - x0 + kAttRows - 1) / kAttRows : 0;
+  int s = 0;
+  if (!issued && warp < nblk) issue(x0 + warp * kAttRows, 0);
   __syncthreads();
 
   // Transposed tile: S^T = K Q^T (M = 16 context rows, N = 8 heads per n tile,

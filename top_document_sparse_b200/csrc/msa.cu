@@ -180,6 +180,7 @@ int attend_splits(int B, int T, int H_kv, int64_t max_ctx) {
 struct AttendPlan {
   int n_split = 1;
   int table_cap = 0;
+  int early = 0;  // the local part may start before the wait for the previous kernel
   size_t part_o = 0, part_ml = 0;  // byte offsets in the workspace
   size_t bytes = 0;
 };
@@ -345,7 +346,7 @@ msa_status launch_attend_mma(const msa_memory *mem, const void *content, const i
       static_cast<__nv_bfloat16 *>(Vc), static_cast<const __nv_bfloat16 *>(K_new),
       static_cast<const __nv_bfloat16 *>(V_new), static_cast<const int32_t *>(cache_len), cap,
       pos_offset, static_cast<const float2 *>(mem->d_rope), scale_log2, plan.n_split,
-      plan.table_cap, fuse_append, static_cast<__nv_bfloat16 *>(O), part_o, part_ml));
+      plan.table_cap, fuse_append, plan.early, static_cast<__nv_bfloat16 *>(O), part_o, part_ml));
   MSA_LAUNCHED("attend_mma_kernel");
   if (plan.n_split > 1) {
     // merge the splits and advance cache_len (every attention CTA has read it)
@@ -385,7 +386,7 @@ msa_status attend_impl(const msa_memory *mem, const void *content, const int32_t
                        const int32_t *slots, int slot_chunks, int B, int k, int T, int H_q,
                        const void *Q, const void *K_new, const void *V_new, void *K_cache,
                        void *V_cache, int32_t *cache_len, int cap, int pos_offset, void *O,
-                       void *ws, size_t ws_bytes, cudaStream_t st) {
+                       void *ws, size_t ws_bytes, cudaStream_t st, bool early = false) {
   if (!mem) return fail(MSA_ERR_INVALID_ARG, "null memory");
   if (B < 1 || T < 1) return fail(MSA_ERR_INVALID_ARG, "batch and tokens must be >= 1");
   if (k < 0 || k > msa::kMaxTopK) return fail(MSA_ERR_INVALID_ARG, "k=%d out of range", k);
@@ -409,7 +410,8 @@ msa_status attend_impl(const msa_memory *mem, const void *content, const int32_t
                 (long long)k * mem->max_doc_chunks, msa::kMaxMemRows);
   if (static_cast<int64_t>(B) * T > 2147483647LL / 64)
     return fail(MSA_ERR_UNSUPPORTED, "batch * tokens too large");
-  const AttendPlan plan = plan_attend(mem, B, T, k, H_q, cap);
+  AttendPlan plan = plan_attend(mem, B, T, k, H_q, cap);
+  plan.early = early ? 1 : 0;
   if (ws_bytes < plan.bytes || (plan.bytes > 0 && !ws))
     return fail(MSA_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, plan.bytes);
   const int D = mem->D, H_kv = mem->H_kv;
@@ -738,9 +740,12 @@ msa_status msa_step(const msa_memory *mem, const void *router_keys, const void *
   msa_status r = route_impl(mem, router_keys, Qr_tok, s->batch, 1, s->top_k, nullptr, s->state,
                             s->ids, s->scores, ws, route_bytes, st);
   if (r != MSA_OK) return r;
+  // the kernel before the attention is the route's top-k, which writes none of cache_len, the
+  // token's Q/K/V or the local cache: the attention may start on its local part early
   return attend_impl(mem, content, s->ids, nullptr, 0, s->batch, s->top_k, 1, s->n_q_heads, Q_tok,
                      K_tok, V_tok, s->k_cache, s->v_cache, s->cache_len, s->cache_capacity,
-                     s->pos_offset, O_tok, ws + route_bytes, s->workspace_bytes - route_bytes, st);
+                     s->pos_offset, O_tok, ws + route_bytes, s->workspace_bytes - route_bytes, st,
+                     /*early=*/true);
 }
 
 msa_status msa_fetcher_create(const msa_memory *mem, const void *content_host, void *slot_cache,
