@@ -220,7 +220,7 @@ RoutePlan plan_route(const msa_memory *mem, int B, int T, int k) {
 // stay resident.
 template <int NT, bool QS = (NT >= 64)>
 msa_status launch_route_tc(const msa_memory *mem, const void *keys, const void *qhat, int R, int T,
-                           float *state, cudaStream_t st) {
+                           float *state, cudaStream_t st, int ctas_per_sm = 1) {
   using L = msa::RouteTcLayout<NT, QS>;
   const int W = mem->H_r * mem->d_r;
   CUtensorMap tmK, tmQ;
@@ -228,8 +228,9 @@ msa_status launch_route_tc(const msa_memory *mem, const void *keys, const void *
   if (s != MSA_OK) return s;
   s = make_map_bf16(&tmQ, qhat, R, W, NT);
   if (s != MSA_OK) return s;
-  const int maxs = max_dyn_smem();
-  int stages = 12;  // (256 B left for the epilogue's static shared memory)
+  // (256 B per CTA left for the epilogue's static shared memory; ~1 KB per CTA reserved)
+  const int maxs = ctas_per_sm == 1 ? max_dyn_smem() : 233472 / ctas_per_sm - 1024 - 256;
+  int stages = 12;
   while (stages > 2 && L::bytes(W, stages) + 256 > static_cast<size_t>(maxs)) --stages;
   const size_t smem = L::bytes(W, stages);
   if (smem + 256 > static_cast<size_t>(maxs))
@@ -240,7 +241,7 @@ msa_status launch_route_tc(const msa_memory *mem, const void *keys, const void *
   const int n_rt = (R + NT - 1) / NT;
   const int64_t n_tiles = static_cast<int64_t>(n_ct) * n_rt;
   if (n_tiles > INT32_MAX) return fail(MSA_ERR_UNSUPPORTED, "too many route tiles");
-  const int grid = static_cast<int>(std::min<int64_t>(n_tiles, num_sms()));
+  const int grid = static_cast<int>(std::min<int64_t>(n_tiles, static_cast<int64_t>(num_sms()) * ctas_per_sm));
   MSA_CUDA(launch_pdl(kern, dim3(grid), dim3(192), smem, st, tmK, tmQ, mem->n_chunks, R, W, T,
                       1.0f / mem->H_r, mem->d_chunk_doc, mem->n_docs, state, n_ct,
                       static_cast<int>(n_tiles), stages));
@@ -299,6 +300,8 @@ msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, i
         s = launch_route_tc<16>(mem, keys, qh, R, T, state, st);
       else if (R <= 32)
         s = launch_route_tc<32>(mem, keys, qh, R, T, state, st);
+      else if (R <= 64)
+        s = launch_route_tc<32, true>(mem, keys, qh, R, T, state, st, 2);
       else
         s = launch_route_tc<64>(mem, keys, qh, R, T, state, st);
       if (s != MSA_OK) return s;
