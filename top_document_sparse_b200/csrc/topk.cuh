@@ -149,34 +149,46 @@ __device__ __forceinline__ void block_select_topk_fast(
   m = warp_sort_desc(m, lane);
   const unsigned long long tw = __shfl_sync(0xffffffffu, m, k - 1);
   if (lane == 0) wt[warp] = tw ? tw : 1ull;
-  if (threadIdx.x == 0) wt[kTopkWarps] = 0ull;  // candidate count
   __syncthreads();
   unsigned long long T = 1ull;
 #pragma unroll
   for (int w = 0; w < kTopkWarps; ++w) T = wt[w] > T ? wt[w] : T;
-  // compact the keys >= T (warp-aggregated slots)
-  unsigned int *count = reinterpret_cast<unsigned int *>(&wt[kTopkWarps]);
+  // compact the keys >= T: per-thread counts, a warp scan and a block prefix
+  // over the warps' totals give every thread its first slot (no atomics)
+  __shared__ unsigned warp_n[kTopkWarps];
+  unsigned c = 0;
 #pragma unroll
-  for (int j = 0; j < kTopkPerThread; ++j) {
-    const bool in = key[j] >= T;
-    const unsigned bal = __ballot_sync(0xffffffffu, in);
-    if (bal == 0u) continue;
-    unsigned base = 0;
-    if (lane == 0) base = atomicAdd(count, static_cast<unsigned>(__popc(bal)));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    const unsigned pos = base + __popc(bal & ((1u << lane) - 1u));
-    if (in && pos < kTopkCandCap) cbuf[pos] = key[j];
+  for (int j = 0; j < kTopkPerThread; ++j) c += key[j] >= T ? 1u : 0u;
+  unsigned inc = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned v = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += v;
   }
+  if (lane == 31) warp_n[warp] = inc;
   __syncthreads();
-  const unsigned n = *count;
-  if (n > kTopkCandCap) {  // uniform: every thread read the same count
+  unsigned n = 0, pos = inc - c;
+#pragma unroll
+  for (int w = 0; w < kTopkWarps; ++w) {
+    const unsigned x = warp_n[w];
+    pos += w < warp ? x : 0u;
+    n += x;
+  }
+  if (n > kTopkCandCap) {  // uniform: every thread summed the same totals
     block_select_topk<KL>(key, k, cand, sel);
     return;
   }
+#pragma unroll
+  for (int j = 0; j < kTopkPerThread; ++j)
+    if (key[j] >= T) cbuf[pos++] = key[j];
+  __syncthreads();
+  // rank by counting: every thread reads the same cbuf entry at once (a
+  // shared-memory broadcast)
   for (unsigned i = threadIdx.x; i < n; i += kTopkThreads) {
     const unsigned long long x = cbuf[i];
     int r = 0;
-    for (unsigned j2 = 0; j2 < n; ++j2) r += cbuf[j2] > x;
+#pragma unroll 8
+    for (unsigned j2 = 0; j2 < n; ++j2) r += cbuf[j2] > x ? 1 : 0;
     if (r < k) sel[r] = x;
   }
   for (int r = static_cast<int>(n) + threadIdx.x; r < k; r += kTopkThreads) sel[r] = 0ull;
@@ -192,8 +204,9 @@ __device__ __forceinline__ void write_topk(const unsigned long long *sel, int k,
   }
 }
 
-// grid (n_split, B).  Warp w of split s holds documents s*kTopkSlice + w*512 +
-// j*32 + lane.  With n_split == 1 the result goes straight to ids/scores.
+// grid (n_split, B).  Warp w of split s holds documents s*kTopkSlice + w*512 ..
+// + 511 (lane l: four runs of 4 from 4 l when the row can be read as float4,
+// else l + 32 j).  With n_split == 1 the result goes straight to ids/scores.
 template <int KL>
 __global__ void __launch_bounds__(kTopkThreads)
 topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__ exclude,
@@ -208,12 +221,29 @@ topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__
   griddep_wait();
   griddep_launch();
   unsigned long long key[kTopkPerThread];
+  const int dw = split * kTopkSlice + warp * (32 * kTopkPerThread);
+  if (exclude == nullptr && (n_docs & 3) == 0 && (reinterpret_cast<uintptr_t>(state) & 15) == 0) {
+    // four 16-byte loads per thread: lane takes documents dw + 128 j4 + 4 lane + 0..3
+    // (n_docs % 4 == 0, so a vector is either wholly inside the row or wholly past it)
 #pragma unroll
-  for (int j = 0; j < kTopkPerThread; ++j) {
-    const int d = split * kTopkSlice + warp * (32 * kTopkPerThread) + j * 32 + lane;
-    bool ok = d < n_docs;
-    if (ok && exclude != nullptr) ok = exclude[row + d] == 0;
-    key[j] = ok ? topk_key(state[row + d], d) : 0ull;
+    for (int j4 = 0; j4 < kTopkPerThread / 4; ++j4) {
+      const int d = dw + j4 * 128 + lane * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (d < n_docs) v = *reinterpret_cast<const float4 *>(state + row + d);
+      const bool ok = d < n_docs;
+      key[4 * j4 + 0] = ok ? topk_key(v.x, d + 0) : 0ull;
+      key[4 * j4 + 1] = ok ? topk_key(v.y, d + 1) : 0ull;
+      key[4 * j4 + 2] = ok ? topk_key(v.z, d + 2) : 0ull;
+      key[4 * j4 + 3] = ok ? topk_key(v.w, d + 3) : 0ull;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kTopkPerThread; ++j) {
+      const int d = dw + j * 32 + lane;
+      bool ok = d < n_docs;
+      if (ok && exclude != nullptr) ok = exclude[row + d] == 0;
+      key[j] = ok ? topk_key(state[row + d], d) : 0ull;
+    }
   }
   block_select_topk_fast<KL>(key, k, wc, sel, wt, cbuf);
   if (n_split == 1) {
