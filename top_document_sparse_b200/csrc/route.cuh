@@ -64,25 +64,24 @@ __device__ __forceinline__ void epi_token_max(float *S, int ldS, int MC, int NR,
   }
 }
 
-// Stage 2 (all nthr threads must call it: it holds named barrier 2): for each
-// (document run inside the tile, query), max over the run's
-// chunks (written over the run's first row of S), then max-merge into state.
-// `segs` (shared, >= MC + 1 ints) receives the run starts.  A run whose document lies wholly inside the chunk tile, for
-// a query whose rows lie wholly inside the row tile, has this CTA as its only
-// writer during the call: it is merged with a plain load / max / store
-// (consecutive threads take consecutive documents, so the accesses coalesce).
-// Runs of documents that straddle a tile edge, and queries split over row
-// tiles, use an atomic float max.
-//   prev_doc / next_doc: document of the chunk just before / after the tile
-//   (-1 at the memory's ends); q_lo / q_hi: the queries whose rows are all
-//   inside the row tile are [q_lo, q_hi) (relative to b0).
-__device__ __forceinline__ void epi_doc_max(float *S, int ldS, int MC, int QB, int64_t b0,
-                                            const int *docs, int prev_doc, int next_doc,
-                                            int q_lo, int q_hi, int n_docs, float *state,
-                                            int *segs, int tid, int nthr, bool write = true) {
-  // run starts by a block-wide ordered compaction (nthr == 128: four warps)
+// Stage 2: for each (document run inside the tile, query), max over the run's
+// chunks, then max-merge into state with an atomic float max.  The atomics
+// are reductions (no value comes back), so the merge costs the CTA no memory
+// round trip; a max is order-independent, so the result is exact and
+// deterministic however the CTAs interleave.  Pieces:
+//   epi_doc_runs     run starts of docs[0..MC) -> segs (ordered compaction)
+//   epi_run_max_smem run maxima of S by columns (any T)
+//   epi_run_max_regs run maxima of register rows by warp shuffles (T == 1)
+//   epi_state_merge  S[run start][q] -> state[b0 + q][doc]
+constexpr int kEpiMaxWarps = 8;
+
+// All nthr (<= 32 * kEpiMaxWarps) threads must call it (named barrier 2);
+// docs[] must be visible to every caller.  Returns the run count; segs[g] is
+// the first row of run g and segs[n_seg] = MC.
+__device__ __forceinline__ int epi_doc_runs(const int *docs, int MC, int *segs, int tid,
+                                            int nthr) {
   const int lane = tid & 31, warp = tid >> 5;
-  __shared__ int warp_cnt[8];
+  __shared__ int warp_cnt[kEpiMaxWarps];
   int n_seg = 0;
   for (int base = 0; base < MC; base += nthr) {
     const int m = base + tid;
@@ -98,10 +97,15 @@ __device__ __forceinline__ void epi_doc_max(float *S, int ldS, int MC, int QB, i
   }
   if (tid == 0) segs[n_seg] = MC;
   asm volatile("bar.sync 2, %0;" ::"r"(nthr) : "memory");
-  // Pass A: run maxima in place -- S[segs[g]][q] = max over run g of column q.
-  // Thread t takes column q = t % QB (consecutive lanes, consecutive banks) and
-  // every (nthr / QB)-th run.  (`write` may differ between threads: every
-  // thread still takes the barrier below.)
+  return n_seg;
+}
+
+// S[segs[g]][q] = max over run g of column q, in place.  Thread t takes column
+// q = t % QB (consecutive lanes, consecutive banks) and every (nthr / QB)-th
+// run.  All nthr threads must call it (named barrier 2); `write` may differ
+// between threads.
+__device__ __forceinline__ void epi_run_max_smem(float *S, int ldS, int QB, const int *segs,
+                                                 int n_seg, int tid, int nthr, bool write) {
   const int cols = QB < nthr ? QB : nthr;
   const int per_col = nthr / cols;
   if (write && tid < cols * per_col) {
@@ -115,55 +119,58 @@ __device__ __forceinline__ void epi_doc_max(float *S, int ldS, int MC, int QB, i
       }
   }
   asm volatile("bar.sync 2, %0;" ::"r"(nthr) : "memory");
-  if (!write) return;  // every thread has passed the barriers above
-  // Pass B: merge into state.  Consecutive threads take consecutive documents
-  // of one query (coalesced).  A thread takes up to kBatch pairs and issues all
-  // their state loads before any store: the pairs are distinct state entries
-  // (a document is one run of the tile), so the loads overlap.  A run whose
-  // document lies wholly inside the chunk tile, for a query whose rows lie
-  // wholly inside the row tile, has this CTA as its only writer during the
-  // call (plain load / max / store); the others use an atomic float max.
-  constexpr int kBatch = 8;
-  const int total = n_seg * QB;
-  for (int p0 = tid; p0 < total; p0 += kBatch * nthr) {
-    float v[kBatch], old[kBatch];
-    float *dst[kBatch];
-    bool plain[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int p = p0 + u * nthr;
-      dst[u] = nullptr;
-      plain[u] = false;
-      if (p < total) {
-        const int q = p / n_seg, g = p - q * n_seg;
-        const int m0 = segs[g], m1 = segs[g + 1];
-        const int d = docs[m0];
-        v[u] = S[m0 * ldS + q];
-        dst[u] = state + (b0 + q) * n_docs + d;
-        const bool whole_doc = (m0 > 0 || prev_doc != d) && (m1 < MC || next_doc != d);
-        plain[u] = whole_doc && q >= q_lo && q < q_hi;
-        if (plain[u]) old[u] = *dst[u];
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      if (dst[u] == nullptr) continue;
-      if (plain[u])
-        *dst[u] = fmaxf(old[u], v[u]);
-      else
-        atomic_max_float(dst[u], v[u]);
-    }
-  }
 }
 
-// Queries (relative to b0 = r0 / T) whose T rows all lie in [r0, r0 + NR).
-__device__ __forceinline__ void query_span(int64_t r0, int NR, int T_tok, int64_t b0, int &q_lo,
-                                           int &q_hi) {
-  const int64_t first_full = (r0 + T_tok - 1) / T_tok;  // first query starting at or after r0
-  const int64_t end_full = (r0 + NR) / T_tok;           // queries ending at or before r0 + NR
-  q_lo = static_cast<int>(first_full - b0);
-  q_hi = static_cast<int>(end_full - b0);
-  if (q_hi < q_lo) q_hi = q_lo;
+// Thread tid holds row tid of the tile's scores in v[0..NC).  Leaves, for every
+// run, its maxima in the run's first row of S (columns 0..NC).  Inside a warp a
+// segmented reduction by shuffles (offsets 1 .. 16: lane l ends up with the max
+// over lanes l .. the end of its run in the warp), whatever a run's length; a
+// run that goes on into later warps then folds in their lane-0 rows.  All nthr
+// threads must call it (named barrier 2); `write` may differ between threads.
+template <int NC>
+__device__ __forceinline__ void epi_run_max_regs(float (&v)[NC], const int *docs, int MC, float *S,
+                                                 int ldS, int tid, int nthr, bool write) {
+  const int lane = tid & 31, warp = tid >> 5;
+  const int m = tid;
+  const int d = m < MC ? docs[m] : -1 - m;  // rows past the tile's chunks: runs of their own
+  const bool start = m == 0 || m >= MC || d != docs[m - 1];
+  const unsigned starts = __ballot_sync(0xffffffffu, start);
+  const unsigned later = lane == 31 ? 0u : starts & (0xffffffffu << (lane + 1));
+  const int run_end = later ? __ffs(later) - 1 : 32;  // first lane past my run in this warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const bool take = lane + o < run_end;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const float t = __shfl_down_sync(0xffffffffu, v[c], o);
+      v[c] = take ? fmaxf(v[c], t) : v[c];
+    }
+  }
+  if (write && m < MC && (start || lane == 0)) {
+#pragma unroll
+    for (int c = 0; c < NC; ++c) S[m * ldS + c] = v[c];
+  }
+  asm volatile("bar.sync 2, %0;" ::"r"(nthr) : "memory");
+  if (write && m < MC && start && run_end == 32) {
+    for (int j = 32 * (warp + 1); j < MC && docs[j] == d; j += 32)
+#pragma unroll
+      for (int c = 0; c < NC; ++c) S[m * ldS + c] = fmaxf(S[m * ldS + c], S[j * ldS + c]);
+  }
+  asm volatile("bar.sync 2, %0;" ::"r"(nthr) : "memory");
+}
+
+// state[b0 + q][doc of run g] = max(itself, S[segs[g]][q]) for every (q < QB,
+// g < n_seg).  Consecutive threads take consecutive runs -- consecutive
+// documents -- of one query, so the reductions coalesce.
+__device__ __forceinline__ void epi_state_merge(const float *S, int ldS, int QB, int64_t b0,
+                                                const int *docs, const int *segs, int n_seg,
+                                                int n_docs, float *state, int tid, int nthr) {
+  const int total = n_seg * QB;
+  for (int p = tid; p < total; p += nthr) {
+    const int q = p / n_seg, g = p - q * n_seg;
+    const int m0 = segs[g];
+    atomic_max_float(state + (b0 + q) * n_docs + docs[m0], S[m0 * ldS + q]);
+  }
 }
 
 // ---------------------------------------------------------------- fp32 path
@@ -206,17 +213,14 @@ route_simt_kernel(const T *__restrict__ Khat, const T *__restrict__ Qhat, int64_
 #pragma unroll
     for (int b = 0; b < 2; ++b) S[(ty + 16 * a) * 33 + tx + 16 * b] = acc[a][b] * inv_Hr;
   if (tid < MC) docs[tid] = chunk_doc[c0 + tid];
-  const int prev_doc = c0 > 0 ? chunk_doc[c0 - 1] : -1;
-  const int next_doc = c0 + MC < C ? chunk_doc[c0 + MC] : -1;
   __syncthreads();
   if (T_tok > 1) epi_token_max(S, 33, MC, NR, r0, T_tok, tid, 256);
   __syncthreads();
   const int64_t b0 = r0 / T_tok;
   const int QB = static_cast<int>((r0 + NR - 1) / T_tok - b0 + 1);
-  int q_lo, q_hi;
-  query_span(r0, NR, T_tok, b0, q_lo, q_hi);
-  epi_doc_max(S, 33, MC, QB, b0, docs, prev_doc, next_doc, q_lo, q_hi, n_docs, state, segs, tid,
-              256);
+  const int n_seg = epi_doc_runs(docs, MC, segs, tid, 256);
+  epi_run_max_smem(S, 33, QB, segs, n_seg, tid, 256, true);
+  epi_state_merge(S, 33, QB, b0, docs, segs, n_seg, n_docs, state, tid, 256);
 }
 
 // ---------------------------------------------------------------- interleave

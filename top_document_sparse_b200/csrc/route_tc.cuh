@@ -14,9 +14,12 @@
 //   warp 5  allocates TMEM; one lane issues 4 UMMAs (K = 16 each) per slice
 //           and commits them to the slice's "empty" barrier, then commits
 //           the finished accumulator to "acc full"
-//   warps 0-3  epilogue: thread t drains TMEM lane t (chunk t of the tile),
-//           scales, then the shared token-max / document-max epilogue with
-//           an atomic max into the running state
+//   warps 0-3  epilogue: while the MMAs run, finds the tile's document runs;
+//           then thread t drains TMEM lane t (chunk t of the tile) into
+//           registers, scales, takes the max over each document run (warp
+//           shuffles; through shared memory after a token max when a query
+//           has several rows) and merges into the running state with atomic
+//           max reductions
 // Two TMEM accumulators alternate, so the epilogue of tile i overlaps the MMAs
 // of tile i+1.  Every barrier wait is bounded; a wait that runs out raises
 // MSA_DEVERR_WAIT_TIMEOUT, later waits are skipped, in-flight copies and MMAs
@@ -195,39 +198,43 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       const int64_t r0 = static_cast<int64_t>(rt) * NT;
       const int MC = static_cast<int>(C - c0 < L::kTileC ? C - c0 : L::kTileC);
       const int NR = static_cast<int>(R - r0 < NT ? R - r0 : NT);
-      // the tile's document ids, loaded while the MMAs run
-      const int my_doc = tid < MC ? chunk_doc[c0 + tid] : 0;
-      const int prev_doc = c0 > 0 ? chunk_doc[c0 - 1] : -1;
-      const int next_doc = c0 + MC < C ? chunk_doc[c0 + MC] : -1;
-      const bool ok = wait(accf0 + 8 * buf, (tl >> 1) & 1);
-      tc05_fence_after();
-      if (ok) {
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) +
-                               static_cast<uint32_t>(buf * NT);
-#pragma unroll
-        for (int c = 0; c < NT; c += 16) {
-          float v[16];
-          tmem_ld16(taddr + c, v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) Sb[tid * L::kLD + c + i] = v[i] * inv_Hr;
-        }
-      }
-      tc05_fence_before();
-      mbar_arrive(acce0 + 8 * buf);  // this accumulator may be overwritten
-      if (tid < MC) docs[tid] = my_doc;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      // after a failed wait the results are void (the error word is set): skip the epilogue
-      const bool go = !*fail;
-      if (go && T_tok > 1) epi_token_max(Sb, L::kLD, MC, NR, r0, T_tok, tid, 128);
-      asm volatile("bar.sync 1, 128;" ::: "memory");
       // (32-bit: r0 + NR <= R, an int)
       const int r0i = static_cast<int>(r0);
       const int b0 = r0i / T_tok;
       const int QB = (r0i + NR - 1) / T_tok - b0 + 1;
-      const int q_lo = (r0i + T_tok - 1) / T_tok - b0;  // queries with all T rows in the tile
-      const int q_hi = max(q_lo, (r0i + NR) / T_tok - b0);
-      epi_doc_max(Sb, L::kLD, MC, QB, b0, docs, prev_doc, next_doc, q_lo, q_hi, n_docs, state,
-                  segs, tid, 128, go);
+      // the tile's documents and their runs, found while the MMAs run
+      if (tid < MC) docs[tid] = chunk_doc[c0 + tid];
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int n_seg = epi_doc_runs(docs, MC, segs, tid, 128);
+      const bool ok = wait(accf0 + 8 * buf, (tl >> 1) & 1);
+      const bool okw = __all_sync(0xffffffffu, ok);
+      tc05_fence_after();
+      float v[NT];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) +
+                             static_cast<uint32_t>(buf * NT);
+#pragma unroll
+      for (int c = 0; c < NT; c += 16) {
+        float x[16];
+        if (okw) tmem_ld16(taddr + c, x);  // (warp-collective: a warp-uniform condition)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[c + i] = okw ? x[i] * inv_Hr : 0.0f;
+      }
+      tc05_fence_before();
+      mbar_arrive(acce0 + 8 * buf);  // this accumulator may be overwritten
+      // after a failed wait the results are void (the error word is set): skip
+      // the writes, but every thread still takes every barrier
+      const bool go = !*fail;
+      if (T_tok == 1) {
+        epi_run_max_regs<NT>(v, docs, MC, Sb, L::kLD, tid, 128, go);
+      } else {
+#pragma unroll
+        for (int c = 0; c < NT; ++c) Sb[tid * L::kLD + c] = v[c];
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (go) epi_token_max(Sb, L::kLD, MC, NR, r0, T_tok, tid, 128);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        epi_run_max_smem(Sb, L::kLD, QB, segs, n_seg, tid, 128, go);
+      }
+      if (go) epi_state_merge(Sb, L::kLD, QB, b0, docs, segs, n_seg, n_docs, state, tid, 128);
       asm volatile("bar.sync 1, 128;" ::: "memory");
     }
   }

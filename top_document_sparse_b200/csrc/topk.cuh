@@ -236,12 +236,17 @@ topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__
       key[4 * j4 + 2] = ok ? topk_key(v.z, d + 2) : 0ull;
       key[4 * j4 + 3] = ok ? topk_key(v.w, d + 3) : 0ull;
     }
+  } else if (exclude == nullptr) {
+#pragma unroll
+    for (int j = 0; j < kTopkPerThread; ++j) {
+      const int d = dw + j * 32 + lane;
+      key[j] = d < n_docs ? topk_key(state[row + d], d) : 0ull;
+    }
   } else {
 #pragma unroll
     for (int j = 0; j < kTopkPerThread; ++j) {
       const int d = dw + j * 32 + lane;
-      bool ok = d < n_docs;
-      if (ok && exclude != nullptr) ok = exclude[row + d] == 0;
+      const bool ok = d < n_docs && exclude[row + d] == 0;
       key[j] = ok ? topk_key(state[row + d], d) : 0ull;
     }
   }
