@@ -14,7 +14,9 @@
 //                         an online softmax (context rows / head dim on M, the
 //                         GQA group's heads on N)
 //   attend_combine_kernel merge context splits (log-sum-exp) and advance
-//                         cache_len
+//                         cache_len (a one-split decode call advances it in
+//                         the attention kernel, whose CTAs of one query form
+//                         a cluster)
 // For a one-token call (decode) the attention kernel appends the new row
 // itself; longer calls run append_kernel first.
 #pragma once
@@ -241,9 +243,9 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
                   const __nv_bfloat16 *__restrict__ Q, int T_tok,
                   __nv_bfloat16 *__restrict__ K_cache, __nv_bfloat16 *__restrict__ V_cache,
                   const __nv_bfloat16 *__restrict__ K_new, const __nv_bfloat16 *__restrict__ V_new,
-                  const int32_t *__restrict__ cache_len, int cap, int pos_offset,
+                  int32_t *__restrict__ cache_len, int cap, int pos_offset,
                   const float2 *__restrict__ rope, float scale_log2, int n_split, int table_cap,
-                  int fuse_append, int early, __nv_bfloat16 *__restrict__ O,
+                  int fuse_append, int early, int cluster_advance, __nv_bfloat16 *__restrict__ O,
                   float *__restrict__ part_o, float *__restrict__ part_ml) {
   constexpr int CPR = D / 8;  // 16-byte chunks per row
   using Sm = AttSmem<D>;
@@ -272,6 +274,10 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
     griddep_launch();
   }
   const int j = (early_ok ? __ldcg(cache_len + b) : cache_len[b]) + i;
+  // cluster_advance (one token, one split, launched as clusters of the query's
+  // H_kv CTAs): this CTA has read cache_len; rank 0 advances it at the end,
+  // after every CTA of the cluster has arrived here
+  if (cluster_advance) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
   const bool overflow = j >= cap || j < 0;
   const int n_loc = overflow ? 0 : j + 1;
   int n_mem = 0, x0 = 0, x1 = n_loc;  // until the table is built, only local rows are issued
@@ -522,6 +528,10 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
         part_ml[(orow * n_split + split) * 2 + 1] = L;
       }
     }
+  }
+  if (cluster_advance) {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    if (g == 0 && threadIdx.x == 0) cache_len[b] = min(j + 1, cap);  // (i == 0: j is the old length)
   }
 }
 

@@ -81,6 +81,27 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// Same, with thread-block clusters of cluster_x CTAs along x (1: none).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                               cudaStream_t st, unsigned cluster_x, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cluster_x > 1 ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Device address of the static attention scratch on the current device, looked
 // up once per device (cudaGetSymbolAddress with that device current).
 msa_status static_attend_scratch(void **out) {
@@ -340,16 +361,22 @@ msa_status launch_attend_mma(const msa_memory *mem, const void *content, const i
   float *part_ml = plan.n_split > 1 ? reinterpret_cast<float *>(wsb + plan.part_ml) : nullptr;
   const float scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)) * 1.4426950408889634);
   const int fuse_append = T == 1 ? 1 : 0;
+  // One token, one split: the H_kv CTAs of a query form a cluster, and the
+  // kernel advances cache_len itself once all of them have read it (cluster
+  // barrier), so no advance kernel follows.
+  const int cluster_advance = (T == 1 && plan.n_split == 1 && mem->H_kv <= 8) ? 1 : 0;
   dim3 grid(static_cast<unsigned>(B * mem->H_kv), plan.n_split, T);
-  MSA_CUDA(launch_pdl(
+  MSA_CUDA(launch_pdl_cluster(
       kern, grid, dim3(32 * msa::kAttWarps), smem, st,
+      static_cast<unsigned>(cluster_advance ? mem->H_kv : 1),
       static_cast<const __nv_bfloat16 *>(content), ids, k,
       static_cast<const int64_t *>(mem->d_doc_chunk_off), mem->n_docs, slots, slot_chunks,
       mem->H_kv, static_cast<const __nv_bfloat16 *>(Q), T, static_cast<__nv_bfloat16 *>(Kc),
       static_cast<__nv_bfloat16 *>(Vc), static_cast<const __nv_bfloat16 *>(K_new),
-      static_cast<const __nv_bfloat16 *>(V_new), static_cast<const int32_t *>(cache_len), cap,
-      pos_offset, static_cast<const float2 *>(mem->d_rope), scale_log2, plan.n_split,
-      plan.table_cap, fuse_append, plan.early, static_cast<__nv_bfloat16 *>(O), part_o, part_ml));
+      static_cast<const __nv_bfloat16 *>(V_new), cache_len, cap, pos_offset,
+      static_cast<const float2 *>(mem->d_rope), scale_log2, plan.n_split, plan.table_cap,
+      fuse_append, plan.early, cluster_advance, static_cast<__nv_bfloat16 *>(O), part_o,
+      part_ml));
   MSA_LAUNCHED("attend_mma_kernel");
   if (plan.n_split > 1) {
     // merge the splits and advance cache_len (every attention CTA has read it)
@@ -359,7 +386,7 @@ msa_status launch_attend_mma(const msa_memory *mem, const void *content, const i
                         static_cast<const float *>(part_ml), plan.n_split, D,
                         static_cast<__nv_bfloat16 *>(O), cache_len, T * mem->H_kv * G, T, cap));
     MSA_LAUNCHED("attend_combine_kernel");
-  } else {
+  } else if (!cluster_advance) {
     MSA_CUDA(launch_pdl(msa::advance_kernel, dim3((B + 255) / 256), dim3(256), 0, st, cache_len, B,
                         T, cap));
     MSA_LAUNCHED("advance_kernel");
