@@ -571,4 +571,237 @@ __global__ void advance_kernel(int32_t *__restrict__ cache_len, int B, int T_tok
   if (b < B) cache_len[b] = min(cache_len[b] + T_tok, cap);
 }
 
+// ---------------------------------------------------------------- bf16 prefill
+// Calls of more than one token: the FlashAttention-2 arrangement.  A warp owns
+// 16 query rows -- 16 / G tokens x the GQA group's G heads -- with Q^T's
+// fragments in registers; the CTA's four warps share every 32-row block of
+// [memory rows in rank order | local rows 0..j_max] staged once in shared
+// memory (two-stage cp.async ring), S = Q K^T and O += P V on mma.sync
+// m16n8k16 with an online softmax per row (log2 units) and the causal mask
+// j <= cache_len + t on local rows.  append_kernel has written the call's new
+// rows before this kernel runs.  grid (B * H_kv, ceil(T / (4 * 16 / G))).
+constexpr int kPfWarps = 4;
+constexpr int kPfRows = 32;  // context rows per block
+
+template <int D>
+struct PfSmem {
+  static constexpr int kBlockBytes = kPfRows * D * 2;  // one K or V block
+  static constexpr int kRing = 2 /*stages*/ * 2 /*K,V*/ * kBlockBytes;
+  static constexpr int kQBytes = kPfWarps * 16 * D * 2;
+  static constexpr int kFixed = kRing + kQBytes + (2 * kMaxTopK + 1) * 4;
+  static int bytes(int table_cap) { return kFixed + table_cap * 4; }
+};
+
+template <int D, int G>
+__global__ void __launch_bounds__(32 * kPfWarps)
+attend_prefill_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__restrict__ ids,
+                      int k, const int64_t *__restrict__ doc_chunk_off, int n_docs,
+                      const int32_t *__restrict__ slots, int slot_chunks, int H_kv,
+                      const __nv_bfloat16 *__restrict__ Q, int T_tok,
+                      const __nv_bfloat16 *__restrict__ K_cache,
+                      const __nv_bfloat16 *__restrict__ V_cache,
+                      const int32_t *__restrict__ cache_len, int cap, int pos_offset,
+                      const float2 *__restrict__ rope, float scale_log2, int table_cap,
+                      __nv_bfloat16 *__restrict__ O) {
+  static_assert(G >= 1 && G <= 16 && 16 % G == 0, "GQA group");
+  constexpr int CPR = D / 8;         // 16-byte chunks per row
+  constexpr int TW = 16 / G;         // tokens per warp
+  constexpr int TC = kPfWarps * TW;  // tokens per CTA
+  constexpr int NTD = D / 8;         // n8 tiles of the output row
+  using Sm = PfSmem<D>;
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint8_t *ring = sm;
+  uint8_t *qsm = sm + Sm::kRing;
+  int *pre = reinterpret_cast<int *>(qsm + Sm::kQBytes);
+  int *base = pre + (kMaxTopK + 1);
+  int *table = base + kMaxTopK;
+
+  const int H_q = H_kv * G;
+  const int b = blockIdx.x / H_kv, g = blockIdx.x % H_kv;
+  const int t0 = blockIdx.y * TC;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t kv = static_cast<int64_t>(H_kv) * D;
+  const int half = D / 2;
+  griddep_wait();
+  griddep_launch();
+  const int len0 = cache_len[b];  // local rows before this call's tokens
+  const int n_mem = build_chunk_table(ids + static_cast<int64_t>(b) * k, k, doc_chunk_off, n_docs,
+                                      slots ? slots + static_cast<int64_t>(b) * k : nullptr,
+                                      slot_chunks, table, pre, base, table_cap);
+  const int t_last = min(t0 + TC, T_tok) - 1;  // last token of the tile
+  const int n_loc = max(0, min(len0 + t_last + 1, cap));
+  const int n_ctx = n_mem + n_loc;
+
+  // rotated query rows -> qsm[warp][16][D]: row r = (token t0 + warp * TW + r / G, head
+  // g * G + r % G); rows of tokens past the call are zero
+  for (int p = threadIdx.x; p < kPfWarps * 16 * half; p += blockDim.x) {
+    const int wr = p / (16 * half), r = (p / half) % 16, e = p % half;
+    const int t = t0 + wr * TW + r / G;
+    float lo = 0.0f, hi = 0.0f;
+    if (t < T_tok && len0 + t < cap) {
+      const __nv_bfloat16 *qr = Q + ((static_cast<int64_t>(b) * T_tok + t) * H_q + g * G + r % G) * D;
+      const float a = __bfloat162float(qr[e]), c = __bfloat162float(qr[e + half]);
+      const float2 cs = rope[static_cast<int64_t>(pos_offset + len0 + t) * half + e];
+      lo = a * cs.x - c * cs.y;
+      hi = c * cs.x + a * cs.y;
+    }
+    uint8_t *qw = qsm + wr * (16 * D * 2);
+    *reinterpret_cast<__nv_bfloat16 *>(qw + swz<D>(r, e / 8) + (e % 8) * 2) = __float2bfloat16_rn(lo);
+    *reinterpret_cast<__nv_bfloat16 *>(qw + swz<D>(r, (e + half) / 8) + (e % 8) * 2) =
+        __float2bfloat16_rn(hi);
+  }
+
+  // the K and V rows of the block at context row x into stage st (one commit)
+  auto issue = [&](int x, int st) {
+    uint8_t *kb = ring + st * 2 * Sm::kBlockBytes;
+#pragma unroll
+    for (int u = 0; u < kPfRows * CPR * 2 / (32 * kPfWarps); ++u) {
+      const int idx = threadIdx.x + 32 * kPfWarps * u;
+      const int which = idx / (kPfRows * CPR), rem = idx % (kPfRows * CPR);
+      const int r = rem / CPR, c = rem % CPR;
+      const int xr = x + r;
+      const bool ok = xr < n_ctx;
+      const __nv_bfloat16 *src = which ? V_cache : K_cache;
+      if (ok) {
+        if (xr < n_mem)
+          src = content + static_cast<int64_t>(table[xr]) * 2 * kv + which * kv + g * D;
+        else
+          src += (static_cast<int64_t>(b) * cap + (xr - n_mem)) * kv + g * D;
+      }
+      cp_async_16(smem_u32(kb + which * Sm::kBlockBytes + swz<D>(r, c)), src + c * 8, ok);
+    }
+    cp_async_commit();
+  };
+  const int nblk = (n_ctx + kPfRows - 1) / kPfRows;
+  if (nblk > 0) issue(0, 0);
+  __syncthreads();  // qsm complete
+
+  // A fragments of this warp's 16 query rows
+  uint32_t qa[D / 16][4];
+  {
+    const uint32_t qbase = smem_u32(qsm + warp * (16 * D * 2));
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk)
+      ldsm_x4(qbase + swz<D>(lane & 15, 2 * kk + (lane >> 4)), qa[kk][0], qa[kk][1], qa[kk][2],
+              qa[kk][3]);
+  }
+  // this thread's two rows: lane / 4 and lane / 4 + 8; the last context row each may see
+  int vis[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int t = t0 + warp * TW + ((lane >> 2) + 8 * h) / G;
+    vis[h] = n_mem + len0 + t;  // context index of local row len0 + t
+  }
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.0f, 0.0f};
+  float o[NTD][4];
+#pragma unroll
+  for (int nt = 0; nt < NTD; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[nt][e] = 0.0f;
+
+  int st = 0;
+  for (int blk = 0; blk < nblk; ++blk) {
+    const int x = blk * kPfRows;
+    if (blk + 1 < nblk) {
+      issue(x + kPfRows, st ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();  // the block is in shared memory for every warp
+    const uint32_t kb = smem_u32(ring + st * 2 * Sm::kBlockBytes);
+    const uint32_t vb = kb + Sm::kBlockBytes;
+    // S = Q K^T: 16 rows x 32 context columns (4 n8 tiles)
+    float sc[kPfRows / 8][4];
+#pragma unroll
+    for (int nt = 0; nt < kPfRows / 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[nt][e] = 0.0f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk)
+#pragma unroll
+      for (int np = 0; np < kPfRows / 16; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kb + swz<D>(16 * np + (lane & 7) + ((lane >> 4) << 3), 2 * kk + ((lane >> 3) & 1)),
+                b0, b1, b2, b3);
+        mma_bf16_16816(sc[2 * np], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
+        mma_bf16_16816(sc[2 * np + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
+      }
+    // online softmax per row; column c of tile nt is context row x + 8 nt + 2 (lane & 3) + e
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float bm = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < kPfRows / 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int xc = x + 8 * nt + 2 * (lane & 3) + e;
+          const bool ok = xc < n_ctx && xc <= vis[h];
+          const float v = ok ? sc[nt][2 * h + e] * scale_log2 : -INFINITY;
+          sc[nt][2 * h + e] = v;
+          bm = fmaxf(bm, v);
+        }
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+      const float mn = fmaxf(mrow[h], bm);
+      // a row that has seen nothing yet (mn = -inf) keeps zero weight and scale 1
+      const float al = mn == -INFINITY ? 1.0f : exp2f(mrow[h] - mn);
+      float ps = 0.0f;
+#pragma unroll
+      for (int nt = 0; nt < kPfRows / 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float pv = mn == -INFINITY ? 0.0f : exp2f(sc[nt][2 * h + e] - mn);
+          sc[nt][2 * h + e] = pv;
+          ps += pv;
+        }
+      mrow[h] = mn;
+      lrow[h] = lrow[h] * al + ps;
+#pragma unroll
+      for (int nt = 0; nt < NTD; ++nt) {
+        o[nt][2 * h] *= al;
+        o[nt][2 * h + 1] *= al;
+      }
+    }
+    // O += P V: P's accumulator pairs are the A fragments of a 16-column k step
+#pragma unroll
+    for (int kk = 0; kk < kPfRows / 16; ++kk) {
+      const uint32_t pa0 = pack_bf16x2(sc[2 * kk][0], sc[2 * kk][1]);
+      const uint32_t pa1 = pack_bf16x2(sc[2 * kk][2], sc[2 * kk][3]);
+      const uint32_t pa2 = pack_bf16x2(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
+      const uint32_t pa3 = pack_bf16x2(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+#pragma unroll
+      for (int dp = 0; dp < D / 16; ++dp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_trans(vb + swz<D>(16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3),
+                                  2 * dp + (lane >> 4)),
+                      b0, b1, b2, b3);
+        mma_bf16_16816(o[2 * dp], pa0, pa1, pa2, pa3, b0, b1);
+        mma_bf16_16816(o[2 * dp + 1], pa0, pa1, pa2, pa3, b2, b3);
+      }
+    }
+    __syncthreads();  // every warp is done with stage st before it is refilled
+    st ^= 1;
+  }
+
+  // row sums over the quad, then O / l for the rows of this call's tokens
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float L = lrow[h];
+    L += __shfl_xor_sync(0xffffffffu, L, 1);
+    L += __shfl_xor_sync(0xffffffffu, L, 2);
+    const int r = (lane >> 2) + 8 * h;
+    const int t = t0 + warp * TW + r / G;
+    if (t >= T_tok) continue;
+    const bool live = len0 + t < cap && L > 0.0f;
+    const float inv = live ? 1.0f / L : 0.0f;
+    __nv_bfloat16 *orow =
+        O + ((static_cast<int64_t>(b) * T_tok + t) * H_q + g * G + r % G) * D + 2 * (lane & 3);
+#pragma unroll
+    for (int nt = 0; nt < NTD; ++nt)
+      *reinterpret_cast<uint32_t *>(orow + 8 * nt) =
+          pack_bf16x2(o[nt][2 * h] * inv, o[nt][2 * h + 1] * inv);
+  }
+}
+
 }  // namespace msa

@@ -352,6 +352,31 @@ msa_status launch_attend_mma(const msa_memory *mem, const void *content, const i
                              const void *Q, const void *K_new, const void *V_new, void *Kc,
                              void *Vc, int32_t *cache_len, int cap, int pos_offset,
                              const AttendPlan &plan, void *O, void *ws, cudaStream_t st) {
+  const float scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)) * 1.4426950408889634);
+  if (T > 1) {
+    // several tokens (prefill): one CTA per (query, kv head, tile of 4 x 16 / G tokens) shares
+    // each staged context block between its tokens; append_kernel ran before
+    using Pf = msa::PfSmem<D>;
+    const int smem_pf = Pf::bytes(plan.table_cap);
+    auto kpf = msa::attend_prefill_kernel<D, G>;
+    MSA_CUDA(cudaFuncSetAttribute(kpf, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_pf));
+    constexpr int TC = msa::kPfWarps * (16 / G);
+    dim3 grid_pf(static_cast<unsigned>(B * mem->H_kv), static_cast<unsigned>((T + TC - 1) / TC));
+    if (grid_pf.y > 65535) return fail(MSA_ERR_UNSUPPORTED, "too many query tokens");
+    MSA_CUDA(launch_pdl(kpf, grid_pf, dim3(32 * msa::kPfWarps), smem_pf, st,
+                        static_cast<const __nv_bfloat16 *>(content), ids, k,
+                        static_cast<const int64_t *>(mem->d_doc_chunk_off), mem->n_docs, slots,
+                        slot_chunks, mem->H_kv, static_cast<const __nv_bfloat16 *>(Q), T,
+                        static_cast<const __nv_bfloat16 *>(Kc), static_cast<const __nv_bfloat16 *>(Vc),
+                        static_cast<const int32_t *>(cache_len), cap, pos_offset,
+                        static_cast<const float2 *>(mem->d_rope), scale_log2, plan.table_cap,
+                        static_cast<__nv_bfloat16 *>(O)));
+    MSA_LAUNCHED("attend_prefill_kernel");
+    MSA_CUDA(launch_pdl(msa::advance_kernel, dim3((B + 255) / 256), dim3(256), 0, st, cache_len, B,
+                        T, cap));
+    MSA_LAUNCHED("advance_kernel");
+    return MSA_OK;
+  }
   using Sm = msa::AttSmem<D>;
   const int smem = Sm::bytes(plan.table_cap);
   auto kern = msa::attend_mma_kernel<D, G>;
@@ -359,8 +384,7 @@ msa_status launch_attend_mma(const msa_memory *mem, const void *content, const i
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   float *part_o = plan.n_split > 1 ? reinterpret_cast<float *>(wsb + plan.part_o) : nullptr;
   float *part_ml = plan.n_split > 1 ? reinterpret_cast<float *>(wsb + plan.part_ml) : nullptr;
-  const float scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)) * 1.4426950408889634);
-  const int fuse_append = T == 1 ? 1 : 0;
+  const int fuse_append = 1;  // (T == 1 here)
   // One token, one split: the H_kv CTAs of a query form a cluster, and the
   // kernel advances cache_len itself once all of them have read it (cluster
   // barrier), so no advance kernel follows.
