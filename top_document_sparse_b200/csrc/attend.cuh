@@ -592,8 +592,9 @@ struct PfSmem {
   static int bytes(int table_cap) { return kFixed + table_cap * 4; }
 };
 
+// (at most 128 registers: four CTAs per SM; measured 5% faster than three at 168)
 template <int D, int G>
-__global__ void __launch_bounds__(32 * kPfWarps)
+__global__ void __launch_bounds__(32 * kPfWarps, 4)
 attend_prefill_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__restrict__ ids,
                       int k, const int64_t *__restrict__ doc_chunk_off, int n_docs,
                       const int32_t *__restrict__ slots, int slot_chunks, int H_kv,

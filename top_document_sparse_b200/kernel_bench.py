@@ -46,7 +46,7 @@ def _graph_time(fn, reps):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="mem1m_bf16")
-    ap.add_argument("--stage", default="all", choices=["all", "route", "topk", "attend"])
+    ap.add_argument("--stage", default="all", choices=["all", "route", "topk", "attend", "prefill"])
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--seed", type=int, default=0)
     a = ap.parse_args(argv)
@@ -104,6 +104,31 @@ def main(argv=None):
         byts = (n_mem + B * (L0 + 1)) * H_kv * 2 * D * 2
         out["attend_us"] = round(t, 2)
         out["attend_gbs"] = round(byts / (t * 1e-6) / 1e9, 1)
+    if a.stage == "prefill":
+        # one layer's multi-token attention: the query's T tokens over [k documents | themselves]
+        T = w.query_tokens
+        ct = torch.randn(mem.n_chunks, 2, H_kv, D, device="cuda", generator=gen).to(torch.bfloat16)
+        ids = torch.from_numpy(np.stack([np.random.default_rng(b).choice(mem.n_docs, k, replace=False)
+                                         for b in range(B)]).astype(np.int32)).cuda()
+        Kc = torch.zeros(B, cap, H_kv, D, dtype=torch.bfloat16, device="cuda")
+        Vc = torch.zeros_like(Kc)
+        Q = torch.randn(B, T, H_q, D, device="cuda", generator=gen).to(torch.bfloat16)
+        Kn = torch.randn(B, T, H_kv, D, device="cuda", generator=gen).to(torch.bfloat16)
+        O = torch.empty_like(Q)
+        clen = torch.zeros(B, dtype=torch.int32, device="cuda")
+        ws = msa.workspace(mem.attend_workspace_size(B, T, k, H_q))
+
+        def pre():
+            clen.zero_()
+            mem.sparse_attend(ct, ids, Q, Kn, Kn, Kc, Vc, clen, k, O, ws)
+
+        t = _graph_time(pre, a.reps)
+        n_mem = np.array([sum(mem.doc_chunk_offsets[d + 1] - mem.doc_chunk_offsets[d] for d in row)
+                          for row in ids.cpu().numpy()], dtype=np.float64)
+        # QK^T and PV over every visible (token, context row) pair: 2 x 2 x D flops each
+        pairs = float(np.sum(n_mem * T + T * (T + 1) / 2)) * H_q
+        out["prefill_us"] = round(t, 2)
+        out["prefill_tflops"] = round(4.0 * D * pairs / (t * 1e-6) / 1e12, 1)
     out["device_error"] = msa.device_error()
     print(json.dumps(out))
 
