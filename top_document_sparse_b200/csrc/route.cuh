@@ -17,11 +17,14 @@ namespace msa {
 // Q_hat[r][h][:] = Q_r[r][h][:] / max(|Q_r[r][h]|, eps).  One CTA per row;
 // thread i owns 4 elements; the d_r/4 threads of a head form an aligned group.
 // Row r = b * T + t of the output reads input row b * pitch + t.
+// The route kernel that follows may start at once: before its own wait it
+// only loads router keys, which no kernel of this library that releases its
+// dependents early ever writes.
 template <typename T>
 __global__ void qnorm_kernel(const T *__restrict__ Qr, int W, int d_r, int T_tok, int pitch,
                              T *__restrict__ out) {
-  griddep_wait();
   griddep_launch();
+  griddep_wait();
   const int64_t r = blockIdx.x;
   const int64_t src_row = (r / T_tok) * pitch + r % T_tok;
   const int e0 = threadIdx.x * 4;

@@ -101,6 +101,30 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   __syncthreads();
   tc05_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The first tile's first key slices are loaded before the wait for the
+  // previous kernel (the query normalisation): router keys are written by no
+  // kernel that can still be running here (see qnorm_kernel).  Query slices,
+  // documents and state come after the wait.
+  int n_pre = 0;
+  if (warp == 4 && lane == 0) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmQ);
+    if (static_cast<int>(blockIdx.x) < n_tiles) {
+      const uint64_t pol = policy_evict_first();
+      const int ct0 = static_cast<int>(blockIdx.x) % n_chunk_tiles;
+      n_pre = stages < KS ? stages : KS;
+      for (int s = 0; s < n_pre; ++s) {
+        // with streamed query slices the stage's arrival (and the query bytes) come after the
+        // wait, so the phase cannot complete on the keys alone
+        if (QS)
+          mbar_expect_tx(full0 + 8 * s, L::kSlice);
+        else
+          mbar_arrive_expect_tx(full0 + 8 * s, L::kStage);
+        tma_load_2d_hint(ks_addr + s * L::kStage, &tmK, 64 * s, ct0 * L::kTileC, full0 + 8 * s,
+                         pol);
+      }
+    }
+  }
   griddep_wait();  // setup above overlaps the previous kernel's drain
   griddep_launch();
 
@@ -115,8 +139,6 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   if (warp == 4) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmQ);
       const uint64_t pol = policy_evict_first();
       int it = 0, qloads = 0, cur_rt = -1;
       for (int tile = blockIdx.x; tile < n_tiles && !*fail; tile += gridDim.x) {
@@ -132,9 +154,13 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         for (int s = 0; s < KS; ++s) {
           const int st = it % stages;
           if (it >= stages && !wait(empty0 + 8 * st, ((it / stages) - 1) & 1)) break;
-          mbar_arrive_expect_tx(full0 + 8 * st, L::kStage);
-          tma_load_2d_hint(ks_addr + st * L::kStage, &tmK, 64 * s, ct * L::kTileC,
-                           full0 + 8 * st, pol);
+          if (it >= n_pre) {
+            mbar_arrive_expect_tx(full0 + 8 * st, L::kStage);
+            tma_load_2d_hint(ks_addr + st * L::kStage, &tmK, 64 * s, ct * L::kTileC,
+                             full0 + 8 * st, pol);
+          } else if (QS) {  // key slice already in flight: arrive with the query bytes
+            mbar_arrive_expect_tx(full0 + 8 * st, L::kQSlice);
+          }
           if (QS)
             tma_load_2d(ks_addr + st * L::kStage + L::kSlice, &tmQ, 64 * s, rt * NT,
                         full0 + 8 * st);
@@ -142,7 +168,10 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         }
       }
       if (*fail) {  // let every copy issued here land before the CTA can exit
-        for (int j = (it > stages ? it - stages : 0); j < it; ++j)
+        if (QS)  // stages whose keys went out early but that the loop never reached
+          for (int j = it; j < n_pre; ++j) mbar_arrive(full0 + 8 * j);
+        const int n_iss = it > n_pre ? it : n_pre;
+        for (int j = (n_iss > stages ? n_iss - stages : 0); j < n_iss; ++j)
           mbar_wait(full0 + 8 * (j % stages), (j / stages) & 1);
         if (qloads > 0) mbar_wait(qfull, (qloads - 1) & 1);
       }
