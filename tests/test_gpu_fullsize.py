@@ -94,6 +94,7 @@ def test_full_size_route_and_decode_on_sampled_outputs(name):
         mem.step(rk, ct, layer, *args)
     torch.cuda.synchronize()
     assert msa.device_error() == 0
+    assert layer.cache_len.cpu().tolist() == [T + 1] * B  # prefill, then one decode token
     ids = layer.ids.cpu().numpy()
     state = to64(layer.state)
 

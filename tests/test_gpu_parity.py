@@ -269,19 +269,32 @@ ATTN_CASES = [
 
 @pytest.mark.parametrize("dt,D,H_q,H_kv,T0,T1,k", ATTN_CASES)
 def test_attend_matches_oracle(dt, D, H_q, H_kv, T0, T1, k):
+    _attend_calls_match_oracle(dt, D, H_q, H_kv, (T0, T1), k, batch=3)
+
+
+def test_one_split_decode_in_clusters_matches_oracle():
+    """A batch with B * H_kv >= 3 CTAs per SM: each one-token call runs with one context split,
+    as clusters of a query's kv-head CTAs that advance cache_len themselves."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    B, H_kv = 64, 8
+    assert B * H_kv >= 3 * sms, "batch too small to take the one-split path on this device"
+    _attend_calls_match_oracle("bf16", 128, 32, H_kv, (6, 1, 1, 1), 3, batch=B)
+
+
+def _attend_calls_match_oracle(dt, D, H_q, H_kv, Ts, k, batch):
     msa = _msa()
     w = small_workload(dtype=dt, head_dim=D, n_q_heads=H_q, n_kv_heads=H_kv, n_docs=0, doc_len=0,
-                       lognormal=(150, 0.8, 3, 600, 5000), batch=3, query_tokens=T0 + T1,
+                       lognormal=(150, 0.8, 3, 600, 5000), batch=batch, query_tokens=sum(Ts),
                        top_k=max(k, 1))
     inp = memory_inputs(w, seed=103 + D + H_q)
-    mem = _build(w, inp, max_local=k + T0 + T1 + 8)
+    mem = _build(w, inp, max_local=k + sum(Ts) + 8)
     rk, ct, _ = _encode(mem, inp)
     Kb, Vb, _ = oracle.encode(inp["K"], inp["V"], inp["Kr"], inp["off"], w.chunk_len, w.rope_theta)
     B = w.batch
     rng = np.random.default_rng(7)
     ids_np = np.stack([rng.choice(mem.n_docs, size=k, replace=False) for _ in range(B)]).astype(np.int32)
     ids = torch.from_numpy(ids_np).cuda() if k else torch.zeros(B, 0, dtype=torch.int32, device="cuda")
-    cap = T0 + T1 + 3
+    cap = sum(Ts) + 3
     dtt = inputs.torch_dtype(dt)
     Kc = torch.zeros(B, cap, H_kv, D, dtype=dtt, device="cuda")
     Vc = torch.zeros_like(Kc)
@@ -290,7 +303,7 @@ def test_attend_matches_oracle(dt, D, H_q, H_kv, T0, T1, k):
     pos_offset = k
     tol = ATTN_TOL[dt]
     start = 0
-    for T in (T0, T1):
+    for T in Ts:
         sl = slice(start, start + T)
         O = torch.empty(B, T, H_q, D, dtype=dtt, device="cuda")
         ws = msa.workspace(mem.attend_workspace_size(B, T, k, H_q))
