@@ -299,7 +299,10 @@ MSA_API msa_status msa_step(const msa_memory *mem, const void *router_keys,
  *   taken  : device [batch][n_docs] uint8, reset to 0 here; on return it marks
  *            every document retrieved in rounds 0..rounds-2
  *   ids, scores : device [rounds][batch][k]
- * The next round's row count is read back to the host once per round.
+ * The next round's row count is read back to the host once per round.  A
+ * query with no new rows in a round (it retrieved nothing) keeps its state
+ * through that round; when no query has new rows, the remaining rounds' ids /
+ * scores are -1 / -inf.
  */
 MSA_API size_t msa_interleave_workspace_size(const msa_memory *mem, int32_t batch,
                                              int32_t tokens, int32_t k);
@@ -308,6 +311,27 @@ MSA_API msa_status msa_interleave(const msa_memory *mem, const void *router_keys
                                   int32_t rounds, float *state, uint8_t *taken, int32_t *ids,
                                   float *scores, void *workspace, size_t workspace_bytes,
                                   msa_stream stream);
+
+/*
+ * Adaptive Memory Interleave [same passages; the pages leave the number of
+ * rounds to the model, which decides when the context holds enough -- here a
+ * stopping score stands in for that decision]: msa_interleave with at most
+ * `max_rounds` rounds, in which a query stops after the first round whose
+ * best new document scores below stop_score.  That round's retrievals do not
+ * enter its context: its ids / scores of that round and every later one are
+ * -1 / -inf, and its state stays as it was after its last kept round.
+ *   n_rounds : device [batch] int32 out, the rounds whose retrievals were kept
+ *              (0 .. max_rounds)
+ *   stop_score : any value but NaN (-inf: never stop = msa_interleave)
+ * Workspace: msa_interleave_workspace_size.  Errors: INVALID_ARG for a null
+ * n_rounds or a NaN stop_score, else as msa_interleave.
+ */
+MSA_API msa_status msa_interleave_adaptive(const msa_memory *mem, const void *router_keys,
+                                           const void *Qr, int32_t batch, int32_t tokens,
+                                           int32_t k, int32_t max_rounds, float stop_score,
+                                           float *state, uint8_t *taken, int32_t *ids,
+                                           float *scores, int32_t *n_rounds, void *workspace,
+                                           size_t workspace_bytes, msa_stream stream);
 
 /*
  * Host tier of the pooled content [Evermind summary sec. 4B "Memory Parallel &

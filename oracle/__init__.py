@@ -222,13 +222,19 @@ def decode_step(state, Qr_tok, Q_tok, K_hist, V_hist, q_index: int, Krbar, Kbar,
     return st, ids, top, O[:, 0]
 
 
-def interleave(Qr, Krbar, doc_chunk_off, k: int, rounds: int):
+def interleave(Qr, Krbar, doc_chunk_off, k: int, rounds: int, stop_score=None):
     """Memory Interleave (retrieval -> context expansion, repeated): each round routes the new
     query rows with the state carried over, takes the top-k among the documents not yet in the
     context, adds them to the context, and appends their pooled router rows (every chunk, every
     head) as the next round's query rows.
 
-    Qr: [B][T][H_r][d_r].  Returns the list of (ids [B][k], top_scores [B][k]) per round."""
+    stop_score (adaptive interleave; the pages leave the round count to the model, a score
+    threshold stands in for its decision): a query whose best new document in a round scores
+    below it stops there -- that round's documents do not enter its context, its ids / scores
+    from that round on are -1 / -inf, and it routes nothing more.
+
+    Qr: [B][T][H_r][d_r].  Returns the list of (ids [B][k], top_scores [B][k]) per round; with
+    stop_score also the final state [B][n_docs] and n_rounds [B] (rounds kept per query)."""
     off = _i64(doc_chunk_off)
     K = f64(Krbar)
     Q = f64(Qr)
@@ -236,16 +242,27 @@ def interleave(Qr, Krbar, doc_chunk_off, k: int, rounds: int):
     n_docs = off.size - 1
     state = np.full((B, n_docs), -np.inf)
     taken = np.zeros((B, n_docs), dtype=bool)
+    active = np.ones(B, dtype=bool)
+    n_rounds = np.zeros(B, dtype=np.int64)
     new_rows = [Q[b] for b in range(B)]
     out = []
     for _ in range(rounds):
         for b in range(B):
-            state[b:b + 1] = route(new_rows[b][None], K, off, state[b:b + 1])
+            if active[b] and new_rows[b].shape[0] > 0:
+                state[b:b + 1] = route(new_rows[b][None], K, off, state[b:b + 1])
         eligible = np.where(taken, -np.inf, state)
         ids, top = topk(eligible, k)
+        if stop_score is not None:
+            active &= top[:, 0] >= stop_score
+            ids[~active] = -1
+            top[~active] = -np.inf
+            n_rounds += active
         out.append((ids, top))
         for b in range(B):
-            taken[b, ids[b]] = True
-        new_rows = [np.concatenate([K[off[d]:off[d + 1]] for d in ids[b]], axis=0)
+            taken[b, ids[b][ids[b] >= 0]] = True
+        new_rows = [np.concatenate([K[off[d]:off[d + 1]] for d in ids[b] if d >= 0] or
+                                   [np.zeros((0,) + K.shape[1:])], axis=0)
                     for b in range(B)]
+    if stop_score is not None:
+        return out, state, n_rounds
     return out

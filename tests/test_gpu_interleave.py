@@ -73,3 +73,50 @@ def test_interleave_k4_retrieves_each_hop_in_its_round():
         o_ids, o_top = ref[0]
         assert chain[b, 0] in o_ids[b]
     assert msa.device_error() == 0
+
+
+@pytest.mark.parametrize("mode,rounds", [("never", 3), ("split", 3), ("chain_end", 4),
+                                         ("always", 3)])
+def test_adaptive_interleave_matches_oracle(mode, rounds):
+    """msa_interleave_adaptive against the oracle's stop rule: a query stops after the first
+    round whose best new document scores below stop_score.  Thresholds: -inf (the fixed rounds),
+    +inf (every query stops after round 0), the midpoint of the widest gap between the per-round
+    best scores (the planted hops score ~0.6 in round 0 and ~0.48 after: stop after round 0's
+    documents), and 0.35 over 4 rounds (keep the three hops, stop on the background).  Every
+    finite threshold is at least 4 x the score tolerance from every decision value, so bf16
+    rounding cannot flip a stop."""
+    msa, w, off, Qr, chain, mem, rk, Krb = _chain_memory(302, "bf16", B=6, T=12,
+                                                          n_docs_lognormal=(200, 1.0, 64, 900, 30000),
+                                                          k=1)
+    tol = 2e-3
+    fixed = oracle.interleave(Qr, Krb, mem.doc_chunk_offsets, k=1, rounds=rounds)
+    vals = np.unique(np.concatenate([r[1][:, 0] for r in fixed]))
+    vals = vals[np.isfinite(vals)]
+    gap, mid = max((vals[i + 1] - vals[i], 0.5 * (vals[i] + vals[i + 1]))
+                   for i in range(vals.size - 1))
+    stop = {"never": -np.inf, "always": np.inf, "split": mid, "chain_end": 0.35}[mode]
+    if np.isfinite(stop):
+        assert np.min(np.abs(vals - stop)) > 4 * tol
+    ids, scores, state, taken, n = mem.interleave_adaptive(rk, Qr.cuda(), k=1, max_rounds=rounds,
+                                                           stop_score=stop)
+    torch.cuda.synchronize()
+    out, st_ref, n_ref = oracle.interleave(Qr, Krb, mem.doc_chunk_offsets, k=1, rounds=rounds,
+                                           stop_score=stop)
+    assert n.cpu().tolist() == n_ref.tolist()
+    got, sc = ids.cpu().numpy(), to64(scores)
+    for r in range(rounds):
+        assert np.array_equal(got[r], out[r][0]), f"round {r}"
+        fin = np.isfinite(out[r][1])
+        assert np.array_equal(np.isfinite(sc[r]), fin)
+        assert np.all(np.abs(sc[r][fin] - out[r][1][fin]) <= tol)
+    st = to64(state)
+    fin = np.isfinite(st_ref)
+    assert np.array_equal(np.isfinite(st), fin)
+    assert np.all(np.abs(st[fin] - st_ref[fin]) <= tol)
+    if mode == "never":
+        assert n_ref.tolist() == [rounds] * 6
+    elif mode == "always":
+        assert n_ref.tolist() == [0] * 6
+    else:  # the threshold stops queries before the last round
+        assert np.all(n_ref < rounds) and np.all(n_ref >= 1)
+    assert msa.device_error() == 0

@@ -376,6 +376,45 @@ def test_interleave_retrieves_planted_chain_hop_by_hop():
         assert len(seen) == 9                             # each round adds new documents
 
 
+def _adaptive_docs():
+    """Four one-chunk documents (H_r = 1, d_r = 4): D0 = e0, D1 = 0.6 e0 + 0.8 e1, D2 = e1,
+    D3 = -e0, and one query token e0.  With k = 1: round 0 takes D0 (cos 1); round 1 routes D0's
+    row (= e0, nothing new) and takes D1 (0.6); round 2 routes D1's row, which raises D2 to 0.8
+    and takes it."""
+    e0, e1 = np.eye(4)[0], np.eye(4)[1]
+    Krb = np.stack([e0, 0.6 * e0 + 0.8 * e1, e1, -e0])[:, None, :]   # [C][H_r][d_r]
+    off = np.arange(5, dtype=np.int64)                                # one chunk per document
+    Qr = e0[None, None, None, :]                                       # [B=1][T=1][H_r][d_r]
+    return Qr, Krb, off
+
+
+def test_adaptive_interleave_stop_rule_on_a_hand_worked_chain():
+    Qr, Krb, off = _adaptive_docs()
+    out, state, n = oracle.interleave(Qr, Krb, off, k=1, rounds=3, stop_score=0.5)
+    assert [int(r[0][0, 0]) for r in out] == [0, 1, 2]
+    np.testing.assert_allclose([r[1][0, 0] for r in out], [1.0, 0.6, 0.8], atol=1e-12)
+    assert n.tolist() == [3]
+    np.testing.assert_allclose(state[0], [1.0, 1.0, 0.8, -0.6], atol=1e-12)  # D3: cos(-e0, D1) = -0.6
+    # 0.7: round 1's best (0.6) is below it -> stop after one kept round; nothing of round 1 or 2
+    out, state, n = oracle.interleave(Qr, Krb, off, k=1, rounds=3, stop_score=0.7)
+    assert [int(r[0][0, 0]) for r in out] == [0, -1, -1]
+    assert np.all(np.isneginf([r[1][0, 0] for r in out[1:]]))
+    assert n.tolist() == [1]
+    np.testing.assert_allclose(state[0], [1.0, 0.6, 0.0, -1.0], atol=1e-12)  # D1's row unrouted
+
+
+def test_adaptive_interleave_limits_reduce_to_fixed_rounds_and_to_round_zero():
+    Qr, Krb, off = _adaptive_docs()
+    fixed = oracle.interleave(Qr, Krb, off, k=2, rounds=3)
+    out, _, n = oracle.interleave(Qr, Krb, off, k=2, rounds=3, stop_score=-np.inf)
+    for (a_ids, a_sc), (b_ids, b_sc) in zip(fixed, out):
+        assert np.array_equal(a_ids, b_ids) and np.array_equal(a_sc, b_sc)
+    assert n.tolist() == [3]
+    out, state, n = oracle.interleave(Qr, Krb, off, k=2, rounds=3, stop_score=np.inf)
+    assert n.tolist() == [0] and all(np.all(r[0] == -1) for r in out)
+    np.testing.assert_allclose(state, oracle.route(Qr, Krb, off), atol=0)  # only round 0 routed
+
+
 # ----------------------------------------------------------------------------- golden example
 def test_golden_hand_worked_example():
     with open(os.path.join(GOLDEN, "hand_worked_route_attend.json")) as f:

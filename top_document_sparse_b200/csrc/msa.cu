@@ -997,11 +997,12 @@ msa_status msa_step_host(const msa_memory *mem, const void *router_keys, msa_fet
                      s->workspace_bytes - route_bytes, st);
 }
 
-// Workspace of msa_interleave: the route workspace for the largest round, the
-// gathered rows [batch][k * max_doc_chunks][W] and the per-query row counts.
+// Workspace of msa_interleave(_adaptive): the route workspace for the largest
+// round, the gathered rows [batch][k * max_doc_chunks][W], the per-query row
+// counts, saved state rows [batch][n_docs] and the active flags [batch].
 struct InterleavePlan {
   int cap = 0;
-  size_t route = 0, rows = 0, count = 0, bytes = 0;
+  size_t route = 0, rows = 0, count = 0, saved = 0, active = 0, bytes = 0;
 };
 
 InterleavePlan plan_interleave(const msa_memory *mem, int B, int T, int k) {
@@ -1012,7 +1013,9 @@ InterleavePlan plan_interleave(const msa_memory *mem, int B, int T, int k) {
   const size_t rb = round256(plan_route(mem, B, std::max(T, p.cap), k).bytes);
   p.rows = rb;
   p.count = p.rows + round256(static_cast<size_t>(B) * p.cap * W * elem_size(mem->dtype));
-  p.bytes = p.count + round256(static_cast<size_t>(B) * 4);
+  p.saved = p.count + round256(static_cast<size_t>(B) * 4);
+  p.active = p.saved + round256(static_cast<size_t>(B) * mem->n_docs * 4);
+  p.bytes = p.active + round256(static_cast<size_t>(B));
   return p;
 }
 
@@ -1022,10 +1025,13 @@ size_t msa_interleave_workspace_size(const msa_memory *mem, int32_t batch, int32
   return plan_interleave(mem, batch, tokens, k).bytes;
 }
 
-msa_status msa_interleave(const msa_memory *mem, const void *router_keys, const void *Qr,
-                          int32_t batch, int32_t tokens, int32_t k, int32_t rounds, float *state,
-                          uint8_t *taken, int32_t *ids, float *scores, void *workspace,
-                          size_t workspace_bytes, msa_stream stream) {
+// Both interleave entry points: adaptive (n_rounds != nullptr) stops a query
+// after the first round whose best new document scores below stop_score.
+static msa_status interleave_impl(const msa_memory *mem, const void *router_keys, const void *Qr,
+                           int32_t batch, int32_t tokens, int32_t k, int32_t rounds,
+                           float stop_score, float *state, uint8_t *taken, int32_t *ids,
+                           float *scores, int32_t *n_rounds, void *workspace,
+                           size_t workspace_bytes, msa_stream stream) {
   if (!mem || !router_keys || !Qr || !state || !taken || !ids || !scores)
     return fail(MSA_ERR_INVALID_ARG, "null argument");
   if (batch < 1 || tokens < 1 || rounds < 1 || k < 1 || k > mem->n_docs || k > msa::kMaxTopK)
@@ -1037,20 +1043,40 @@ msa_status msa_interleave(const msa_memory *mem, const void *router_keys, const 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   void *rows = ws + plan.rows;
   int32_t *count = reinterpret_cast<int32_t *>(ws + plan.count);
+  float *saved = reinterpret_cast<float *>(ws + plan.saved);
+  uint8_t *active = ws + plan.active;
   const int W = mem->H_r * mem->d_r;
   const int64_t nd = static_cast<int64_t>(batch) * mem->n_docs;
   msa_status r = msa_route_reset(state, nd, stream);
   if (r != MSA_OK) return r;
   MSA_CUDA(cudaMemsetAsync(taken, 0, static_cast<size_t>(nd), st));
+  if (n_rounds) {
+    MSA_CUDA(cudaMemsetAsync(active, 1, static_cast<size_t>(batch), st));
+    MSA_CUDA(cudaMemsetAsync(n_rounds, 0, static_cast<size_t>(batch) * sizeof(int32_t), st));
+  }
   const void *q = Qr;
   int T = tokens;
+  bool hold = false;  // some query has no new rows this round
   std::vector<int32_t> h_count(batch);
   for (int round = 0; round < rounds; ++round) {
     int32_t *ids_r = ids + static_cast<int64_t>(round) * batch * k;
     float *sc_r = scores + static_cast<int64_t>(round) * batch * k;
+    if (hold) {
+      msa::hold_state_kernel<<<batch, 256, 0, st>>>(state, saved, count, mem->n_docs, 0);
+      MSA_LAUNCHED("hold_state_kernel");
+    }
     r = route_impl(mem, router_keys, q, batch, T, k, taken, state, ids_r, sc_r, ws, plan.rows, st,
                    q == Qr ? T : plan.cap);
     if (r != MSA_OK) return r;
+    if (hold) {
+      msa::hold_state_kernel<<<batch, 256, 0, st>>>(state, saved, count, mem->n_docs, 1);
+      MSA_LAUNCHED("hold_state_kernel");
+    }
+    if (n_rounds) {
+      msa::interleave_stop_kernel<<<(batch + 127) / 128, 128, 0, st>>>(
+          ids_r, sc_r, batch, k, stop_score, active, n_rounds, round);
+      MSA_LAUNCHED("interleave_stop_kernel");
+    }
     if (round + 1 == rounds) break;
     if (mem->dtype == MSA_BF16) {
       msa::gather_rows_kernel<__nv_bfloat16><<<batch, 256, 0, st>>>(
@@ -1066,8 +1092,23 @@ msa_status msa_interleave(const msa_memory *mem, const void *router_keys, const 
                              cudaMemcpyDeviceToHost, st));
     MSA_CUDA(cudaStreamSynchronize(st));
     int T_next = 0;
-    for (int b = 0; b < batch; ++b) T_next = std::max(T_next, static_cast<int>(h_count[b]));
-    if (T_next == 0) T_next = 1;  // nothing retrieved: route one (zero) row
+    hold = false;
+    for (int b = 0; b < batch; ++b) {
+      T_next = std::max(T_next, static_cast<int>(h_count[b]));
+      hold = hold || h_count[b] == 0;
+    }
+    if (T_next == 0) {
+      // no query has new rows: the remaining rounds retrieve nothing
+      for (int rr = round + 1; rr < rounds; ++rr) {
+        MSA_CUDA(cudaMemsetAsync(ids + static_cast<int64_t>(rr) * batch * k, 0xFF,
+                                 static_cast<size_t>(batch) * k * sizeof(int32_t), st));
+        const int64_t n = static_cast<int64_t>(batch) * k;
+        msa::fill_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+            scores + static_cast<int64_t>(rr) * batch * k, n, -INFINITY);
+        MSA_LAUNCHED("fill_kernel");
+      }
+      break;
+    }
     if (mem->dtype == MSA_BF16) {
       msa::pad_rows_kernel<__nv_bfloat16><<<batch, 256, 0, st>>>(
           static_cast<__nv_bfloat16 *>(rows), plan.cap, W, count, T_next);
@@ -1081,6 +1122,26 @@ msa_status msa_interleave(const msa_memory *mem, const void *router_keys, const 
     T = T_next;
   }
   return MSA_OK;
+}
+
+msa_status msa_interleave(const msa_memory *mem, const void *router_keys, const void *Qr,
+                          int32_t batch, int32_t tokens, int32_t k, int32_t rounds, float *state,
+                          uint8_t *taken, int32_t *ids, float *scores, void *workspace,
+                          size_t workspace_bytes, msa_stream stream) {
+  return interleave_impl(mem, router_keys, Qr, batch, tokens, k, rounds, -INFINITY, state, taken,
+                         ids, scores, nullptr, workspace, workspace_bytes, stream);
+}
+
+msa_status msa_interleave_adaptive(const msa_memory *mem, const void *router_keys,
+                                   const void *Qr, int32_t batch, int32_t tokens, int32_t k,
+                                   int32_t max_rounds, float stop_score, float *state,
+                                   uint8_t *taken, int32_t *ids, float *scores,
+                                   int32_t *n_rounds, void *workspace, size_t workspace_bytes,
+                                   msa_stream stream) {
+  if (!n_rounds) return fail(MSA_ERR_INVALID_ARG, "null n_rounds");
+  if (stop_score != stop_score) return fail(MSA_ERR_INVALID_ARG, "stop_score is NaN");
+  return interleave_impl(mem, router_keys, Qr, batch, tokens, k, max_rounds, stop_score, state,
+                         taken, ids, scores, n_rounds, workspace, workspace_bytes, stream);
 }
 
 msa_status msa_device_error(uint32_t *bits, msa_stream stream) {

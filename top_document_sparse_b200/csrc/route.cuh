@@ -270,7 +270,13 @@ __global__ void pad_rows_kernel(T *__restrict__ rows, int cap, int W,
                                 const int32_t *__restrict__ count, int T_rows) {
   const int b = blockIdx.x;
   const int n = count[b];
-  if (n <= 0 || n >= T_rows) return;
+  if (n <= 0) {  // no new rows: zero rows (their state row is saved and restored around the route)
+    const int64_t total = static_cast<int64_t>(T_rows) * W;
+    for (int64_t i = threadIdx.x; i < total; i += blockDim.x)
+      rows[static_cast<int64_t>(b) * cap * W + i] = Elem<T>::from_f(0.0f);
+    return;
+  }
+  if (n >= T_rows) return;
   const T *src = rows + static_cast<int64_t>(b) * cap * W;
   const int64_t per = W / 4;
   const int64_t total = static_cast<int64_t>(T_rows - n) * per;
@@ -279,6 +285,47 @@ __global__ void pad_rows_kernel(T *__restrict__ rows, int cap, int W,
     float v[4];
     load4(src + e, v);
     store4(rows + (static_cast<int64_t>(b) * cap + row) * W + e, v);
+  }
+}
+
+// grid (B): for the queries with no new rows this round (count[b] == 0), copy
+// state row b to saved (dir 0, before the route) or back (dir 1, after it), so
+// that routing their padding rows leaves their running state as it was.
+__global__ void hold_state_kernel(float *__restrict__ state, float *__restrict__ saved,
+                                  const int32_t *__restrict__ count, int n_docs, int dir) {
+  const int b = blockIdx.x;
+  if (count[b] != 0) return;
+  float *st = state + static_cast<int64_t>(b) * n_docs;
+  float *sv = saved + static_cast<int64_t>(b) * n_docs;
+  for (int d = threadIdx.x; d < n_docs; d += blockDim.x) {
+    if (dir == 0)
+      sv[d] = st[d];
+    else
+      st[d] = sv[d];
+  }
+}
+
+// Adaptive Memory Interleave, after round r's top-k (one thread per query): a
+// query still active whose best new document scores below stop_score stops
+// (active[b] = 0); a stopped query's ids / scores of this round become -1 /
+// -inf (nothing of the round enters its context); an active one records
+// n_rounds[b] = r + 1.
+__global__ void interleave_stop_kernel(int32_t *__restrict__ ids, float *__restrict__ scores,
+                                       int B, int k, float stop_score,
+                                       uint8_t *__restrict__ active, int32_t *__restrict__ n_rounds,
+                                       int round) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  int32_t *id = ids + static_cast<int64_t>(b) * k;
+  float *sc = scores + static_cast<int64_t>(b) * k;
+  if (active[b] && !(sc[0] >= stop_score)) active[b] = 0;  // (a -inf best score stops too)
+  if (active[b]) {
+    n_rounds[b] = round + 1;
+    return;
+  }
+  for (int r = 0; r < k; ++r) {
+    id[r] = -1;
+    sc[r] = -INFINITY;
   }
 }
 

@@ -90,6 +90,8 @@ SIGNATURES = {
     "msa_interleave_workspace_size": (_SZ, [_P, _I32, _I32, _I32]),
     "msa_interleave": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ,
                                       _P]),
+    "msa_interleave_adaptive": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, ctypes.c_float,
+                                               _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "msa_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "msa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "msa_last_error": (ctypes.c_char_p, []),
@@ -261,6 +263,24 @@ class Memory:
                                    _ptr(state), _ptr(taken), _ptr(ids), _ptr(scores), _ptr(ws),
                                    ws.numel(), _stream(stream)))
         return ids, scores, state, taken
+
+    def interleave_adaptive(self, router_keys, Qr, k: int, max_rounds: int, stop_score: float,
+                            stream=None):
+        """Adaptive Memory Interleave (msa_interleave_adaptive): returns (ids [max_rounds][B][k],
+        scores, state [B][n_docs], taken [B][n_docs], n_rounds [B])."""
+        B, T = Qr.shape[0], Qr.shape[1]
+        dev = Qr.device
+        state = torch.empty(B, self.n_docs, dtype=torch.float32, device=dev)
+        taken = torch.empty(B, self.n_docs, dtype=torch.uint8, device=dev)
+        ids = torch.empty(max_rounds, B, k, dtype=torch.int32, device=dev)
+        scores = torch.empty(max_rounds, B, k, dtype=torch.float32, device=dev)
+        n_rounds = torch.empty(B, dtype=torch.int32, device=dev)
+        ws = workspace(_lib.msa_interleave_workspace_size(self.handle, B, T, k), dev)
+        _check(_lib.msa_interleave_adaptive(self.handle, _ptr(router_keys), _ptr(Qr), B, T, k,
+                                            max_rounds, float(stop_score), _ptr(state),
+                                            _ptr(taken), _ptr(ids), _ptr(scores), _ptr(n_rounds),
+                                            _ptr(ws), ws.numel(), _stream(stream)))
+        return ids, scores, state, taken, n_rounds
 
     def step_workspace_size(self, batch: int, k: int, n_q_heads: int) -> int:
         return _lib.msa_step_workspace_size(self.handle, batch, k, n_q_heads)
