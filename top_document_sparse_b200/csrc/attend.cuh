@@ -214,6 +214,12 @@ attend_simt_kernel(const T *__restrict__ content, const int32_t *__restrict__ id
 // CTAs share an SM, so the 8 x 64 (query, kv head) CTAs of a decode batch run in one wave.
 constexpr int kAttWarps = 3;
 constexpr int kAttRows = 16;  // context rows per warp block
+// Early path: local blocks past the ring's first that a warp prefetches into L2
+// while the previous kernel (the top-k, which leaves HBM idle) finishes.
+#ifndef MSA_ATT_EARLY_L2
+#define MSA_ATT_EARLY_L2 2
+#endif
+constexpr int kAttEarlyL2 = MSA_ATT_EARLY_L2;
 
 template <int D>
 struct AttSmem {
@@ -337,6 +343,16 @@ attend_mma_kernel(const __nv_bfloat16 *__restrict__ content, const int32_t *__re
   if (early_ok && (warp + 1) * kAttRows <= n_loc) {
     issue(warp * kAttRows, 0);
     issued = true;
+    // and the warp's next all-local blocks into L2: lane l takes row l / 2 of K (l even) or V
+#pragma unroll 1
+    for (int p = 1; p <= kAttEarlyL2; ++p) {
+      const int x = (warp + p * kAttWarps) * kAttRows;
+      if (x + kAttRows > n_loc) break;
+      const __nv_bfloat16 *src = ((lane & 1) ? V_cache : K_cache) +
+                                 (static_cast<int64_t>(b) * cap + x + (lane >> 1)) * kv + g * D;
+#pragma unroll
+      for (int o = 0; o < D * 2; o += 128) prefetch_l2(reinterpret_cast<const uint8_t *>(src) + o);
+    }
   }
   // rotated query rows of the group -> qsm [16][D] (rows >= G are zero)
   {

@@ -129,6 +129,11 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Prefetch the 128-byte line holding `p` into L2 (no data reaches the SM).
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialization may start while the kernel before it on the stream drains;
 // griddep_wait() blocks until that kernel has completed and its memory is
