@@ -323,8 +323,10 @@ msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, i
         s = launch_route_tc<32>(mem, keys, qh, R, T, state, st);
       else if (R <= 64)
         s = launch_route_tc<32, true>(mem, keys, qh, R, T, state, st, 2);
-      else
+      else if (R <= 128)
         s = launch_route_tc<64>(mem, keys, qh, R, T, state, st);
+      else  // many rows (prefill, interleave rounds): 128-row tiles re-read each key slice half as often
+        s = launch_route_tc<128, true>(mem, keys, qh, R, T, state, st);
       if (s != MSA_OK) return s;
     } else {
       auto *qh = reinterpret_cast<float *>(wsb + plan.qhat);

@@ -61,6 +61,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 int n_chunk_tiles, int n_tiles, int stages) {
   using L = RouteTcLayout<NT, QS>;
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "UMMA N");
+  constexpr bool kRegRuns = NT <= 64;  // document-run max in registers (one-token rows)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -238,31 +239,47 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       const bool ok = wait(accf0 + 8 * buf, (tl >> 1) & 1);
       const bool okw = __all_sync(0xffffffffu, ok);
       tc05_fence_after();
-      float v[NT];
       const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) +
                              static_cast<uint32_t>(buf * NT);
+      // After a failed wait the results are void (the error word is set): the
+      // writes are skipped (`go`), but every thread still takes every barrier.
+      // Shared-memory path: staged 16 columns at a time, token max, run max by columns.
+      auto staged = [&]() {
+#pragma unroll 4
+        for (int c = 0; c < NT; c += 16) {
+          float x[16];
+          if (okw) tmem_ld16(taddr + c, x);  // (warp-collective: a warp-uniform condition)
 #pragma unroll
-      for (int c = 0; c < NT; c += 16) {
-        float x[16];
-        if (okw) tmem_ld16(taddr + c, x);  // (warp-collective: a warp-uniform condition)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[c + i] = okw ? x[i] * inv_Hr : 0.0f;
-      }
-      tc05_fence_before();
-      mbar_arrive(acce0 + 8 * buf);  // this accumulator may be overwritten
-      // after a failed wait the results are void (the error word is set): skip
-      // the writes, but every thread still takes every barrier
-      const bool go = !*fail;
-      if (T_tok == 1) {
-        epi_run_max_regs<NT>(v, docs, MC, Sb, L::kLD, tid, 128, go);
-      } else {
-#pragma unroll
-        for (int c = 0; c < NT; ++c) Sb[tid * L::kLD + c] = v[c];
+          for (int i = 0; i < 16; ++i) Sb[tid * L::kLD + c + i] = okw ? x[i] * inv_Hr : 0.0f;
+        }
+        tc05_fence_before();
+        mbar_arrive(acce0 + 8 * buf);  // this accumulator may be overwritten
+        const bool go = !*fail;
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (go) epi_token_max(Sb, L::kLD, MC, NR, r0, T_tok, tid, 128);
+        if (go && T_tok > 1) epi_token_max(Sb, L::kLD, MC, NR, r0, T_tok, tid, 128);
         asm volatile("bar.sync 1, 128;" ::: "memory");
         epi_run_max_smem(Sb, L::kLD, QB, segs, n_seg, tid, 128, go);
+      };
+      if constexpr (kRegRuns) {
+        if (T_tok == 1) {  // one token per query: the run max in registers
+          float v[NT];
+#pragma unroll
+          for (int c = 0; c < NT; c += 16) {
+            float x[16];
+            if (okw) tmem_ld16(taddr + c, x);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[c + i] = okw ? x[i] * inv_Hr : 0.0f;
+          }
+          tc05_fence_before();
+          mbar_arrive(acce0 + 8 * buf);  // this accumulator may be overwritten
+          epi_run_max_regs<NT>(v, docs, MC, Sb, L::kLD, tid, 128, !*fail);
+        } else {
+          staged();
+        }
+      } else {
+        staged();
       }
+      const bool go = !*fail;
       if (go) epi_state_merge(Sb, L::kLD, QB, b0, docs, segs, n_seg, n_docs, state, tid, 128);
       asm volatile("bar.sync 1, 128;" ::: "memory");
     }
