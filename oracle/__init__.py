@@ -252,6 +252,11 @@ def interleave(Qr, Krbar, doc_chunk_off, k: int, rounds: int, stop_score=None):
                 state[b:b + 1] = route(new_rows[b][None], K, off, state[b:b + 1])
         eligible = np.where(taken, -np.inf, state)
         ids, top = topk(eligible, k)
+        # a document already in the context cannot be retrieved again: with fewer than k
+        # eligible documents the round's list is padded with -1 / -inf
+        excluded = np.take_along_axis(taken, ids.astype(np.int64), axis=1)
+        ids[excluded] = -1
+        top[excluded] = -np.inf
         if stop_score is not None:
             active &= top[:, 0] >= stop_score
             ids[~active] = -1

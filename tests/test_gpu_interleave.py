@@ -120,3 +120,46 @@ def test_adaptive_interleave_matches_oracle(mode, rounds):
     else:  # the threshold stops queries before the last round
         assert np.all(n_ref < rounds) and np.all(n_ref >= 1)
     assert msa.device_error() == 0
+
+
+def test_interleave_when_queries_run_out_of_documents():
+    """A memory of 3 documents, k = 1, 5 rounds: the last two rounds have nothing eligible left,
+    so their ids / scores are -1 / -inf, and a query with no new rows keeps its state."""
+    from top_document_sparse_b200 import msa
+    from helpers import small_workload as sw
+    w = sw(n_docs=3, doc_len=128, batch=2, query_tokens=4, top_k=1)
+    off = inputs.doc_offsets(w, 5)
+    K, V, Kr = inputs.raw_memory(w, int(off[-1]), 5)
+    Qr, _, _, _ = inputs.queries(w, 2, 4, 6)
+    mem = msa.Memory(off, w.chunk_len, w.n_kv_heads, w.head_dim, w.n_router_heads, w.router_dim,
+                     inputs.torch_dtype(w.dtype), w.rope_theta, 16)
+    rk, ct = mem.new_router_keys(), mem.new_content()
+    mem.encode(0, mem.n_docs, K.cuda(), V.cuda(), Kr.cuda(), rk, ct)
+    torch.cuda.synchronize()
+    _, _, Krb = oracle.encode(K, V, Kr, off, w.chunk_len, w.rope_theta)
+    ids, scores, state, taken = mem.interleave(rk, Qr.cuda(), k=1, rounds=5)
+    torch.cuda.synchronize()
+    ref = oracle.interleave(Qr, Krb, mem.doc_chunk_offsets, k=1, rounds=5)
+    got = ids.cpu().numpy()
+    for r in range(5):
+        fin = np.isfinite(ref[r][1])
+        # rounds 0-2: each query takes the three documents one by one; the ranking is the oracle's
+        # wherever its top two scores are apart (bf16 keys); rounds 3-4: nothing left
+        if r >= 3:
+            assert np.all(got[r] == -1) and np.all(ref[r][0] == -1)
+            assert np.all(np.isneginf(to64(scores[r])))
+        else:
+            assert np.all(fin) and np.all(got[r] >= 0)
+    assert all(sorted(got[:3, b, 0].tolist()) == [0, 1, 2] for b in range(2))
+    assert np.all(taken.cpu().numpy() == 1)
+    # the state after the last routed round (round 3 routes round 2's document; round 4 has no
+    # rows) is the oracle's, whatever the order of the picks
+    if np.array_equal(got[:3], np.stack([r[0] for r in ref[:3]])):
+        st, st_ref = to64(state), oracle.route(Qr, Krb, mem.doc_chunk_offsets)
+        for r in range(3):
+            rows = [np.concatenate([Krb[mem.doc_chunk_offsets[d]:mem.doc_chunk_offsets[d + 1]]
+                                    for d in got[r, b]])[None] for b in range(2)]
+            st_ref = np.concatenate([oracle.route(rows[b], Krb, mem.doc_chunk_offsets,
+                                                  st_ref[b:b + 1]) for b in range(2)])
+        assert np.all(np.abs(st - st_ref) <= 2e-3)
+    assert msa.device_error() == 0

@@ -415,6 +415,14 @@ def test_adaptive_interleave_limits_reduce_to_fixed_rounds_and_to_round_zero():
     np.testing.assert_allclose(state, oracle.route(Qr, Krb, off), atol=0)  # only round 0 routed
 
 
+def test_interleave_pads_with_minus_one_once_every_document_is_in_the_context():
+    Qr, Krb, off = _adaptive_docs()                     # four documents, k = 1
+    out = oracle.interleave(Qr, Krb, off, k=1, rounds=6)
+    ids = [int(r[0][0, 0]) for r in out]
+    assert sorted(ids[:4]) == [0, 1, 2, 3] and ids[4:] == [-1, -1]
+    assert all(np.isneginf(r[1][0, 0]) for r in out[4:])
+
+
 # ----------------------------------------------------------------------------- golden example
 def test_golden_hand_worked_example():
     with open(os.path.join(GOLDEN, "hand_worked_route_attend.json")) as f:
