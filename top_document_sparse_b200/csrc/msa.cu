@@ -274,8 +274,13 @@ template <int KL>
 msa_status launch_topk(const msa_memory *mem, const float *state, const uint8_t *exclude, int B,
                        int k, int n_split, unsigned long long *cand, int32_t *ids, float *scores,
                        cudaStream_t st) {
-  MSA_CUDA(launch_pdl(msa::topk_partial_kernel<KL>, dim3(n_split, B), dim3(msa::kTopkThreads), 0,
-                      st, state, exclude, mem->n_docs, k, n_split, cand, ids, scores));
+  if (n_split == 1 && mem->n_docs <= 128 * msa::kTopkPerThread) {
+    MSA_CUDA(launch_pdl(msa::topk_partial_kernel<KL, 128>, dim3(1, B), dim3(128), 0, st, state,
+                        exclude, mem->n_docs, k, 1, cand, ids, scores));
+  } else {
+    MSA_CUDA(launch_pdl(msa::topk_partial_kernel<KL>, dim3(n_split, B), dim3(msa::kTopkThreads),
+                        0, st, state, exclude, mem->n_docs, k, n_split, cand, ids, scores));
+  }
   MSA_LAUNCHED("topk_partial_kernel");
   if (n_split > 1) {
     MSA_CUDA(launch_pdl(msa::topk_merge_kernel<KL>, dim3(B), dim3(msa::kTopkThreads), 0, st,

@@ -78,8 +78,9 @@ __device__ __forceinline__ void merge_with_lane(unsigned long long (&a)[KL], int
 
 // Block top-k (k <= KL) of the threads' key[] registers (kTopkPerThread each):
 // per-lane sort, warp butterflies, then warp 0 merges the warps' lists.  The
-// k largest keys, descending, end in sel[0..k).
-template <int KL>
+// k largest keys, descending, end in sel[0..k).  NTHR: the block's threads (a
+// multiple of 32, at most 1024); cand holds NTHR / 32 lists of KL keys.
+template <int KL, int NTHR = kTopkThreads>
 __device__ __forceinline__ void block_select_topk(const unsigned long long (&key)[kTopkPerThread],
                                                   int k, unsigned long long *cand,
                                                   unsigned long long *sel) {
@@ -96,10 +97,12 @@ __device__ __forceinline__ void block_select_topk(const unsigned long long (&key
   }
   __syncthreads();
   if (warp == 0) {
+    constexpr int NW = NTHR / 32;
+    constexpr int NWP = NW <= 1 ? 1 : NW <= 2 ? 2 : NW <= 4 ? 4 : NW <= 8 ? 8 : NW <= 16 ? 16 : 32;
 #pragma unroll
-    for (int i = 0; i < KL; ++i) a[i] = lane < kTopkWarps ? cand[lane * KL + i] : 0ull;
+    for (int i = 0; i < KL; ++i) a[i] = lane < NW ? cand[lane * KL + i] : 0ull;
 #pragma unroll
-    for (int o = kTopkWarps >> 1; o > 0; o >>= 1) merge_with_lane<KL>(a, o);
+    for (int o = NWP >> 1; o > 0; o >>= 1) merge_with_lane<KL>(a, o);
     if (lane == 0)
       for (int i = 0; i < k; ++i) sel[i] = a[i];
   }
@@ -132,14 +135,15 @@ __device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long 
   return v;
 }
 
-// Same contract as block_select_topk.  Shared scratch: wt[kTopkWarps + 1] and
+// Same contract as block_select_topk.  Shared scratch: wt[NTHR / 32] and
 // cbuf[kTopkCandCap] besides block_select_topk's.
-template <int KL>
+template <int KL, int NTHR = kTopkThreads>
 __device__ __forceinline__ void block_select_topk_fast(
     const unsigned long long (&key)[kTopkPerThread], int k, unsigned long long *cand,
     unsigned long long *sel, unsigned long long *wt, unsigned long long *cbuf) {
+  constexpr int NW = NTHR / 32;
   if (k > 32) {
-    block_select_topk<KL>(key, k, cand, sel);
+    block_select_topk<KL, NTHR>(key, k, cand, sel);
     return;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -152,10 +156,10 @@ __device__ __forceinline__ void block_select_topk_fast(
   __syncthreads();
   unsigned long long T = 1ull;
 #pragma unroll
-  for (int w = 0; w < kTopkWarps; ++w) T = wt[w] > T ? wt[w] : T;
+  for (int w = 0; w < NW; ++w) T = wt[w] > T ? wt[w] : T;
   // compact the keys >= T: per-thread counts, a warp scan and a block prefix
   // over the warps' totals give every thread its first slot (no atomics)
-  __shared__ unsigned warp_n[kTopkWarps];
+  __shared__ unsigned warp_n[NW];
   unsigned c = 0;
 #pragma unroll
   for (int j = 0; j < kTopkPerThread; ++j) c += key[j] >= T ? 1u : 0u;
@@ -169,13 +173,13 @@ __device__ __forceinline__ void block_select_topk_fast(
   __syncthreads();
   unsigned n = 0, pos = inc - c;
 #pragma unroll
-  for (int w = 0; w < kTopkWarps; ++w) {
+  for (int w = 0; w < NW; ++w) {
     const unsigned x = warp_n[w];
     pos += w < warp ? x : 0u;
     n += x;
   }
   if (n > kTopkCandCap) {  // uniform: every thread summed the same totals
-    block_select_topk<KL>(key, k, cand, sel);
+    block_select_topk<KL, NTHR>(key, k, cand, sel);
     return;
   }
 #pragma unroll
@@ -184,20 +188,21 @@ __device__ __forceinline__ void block_select_topk_fast(
   __syncthreads();
   // rank by counting: every thread reads the same cbuf entry at once (a
   // shared-memory broadcast)
-  for (unsigned i = threadIdx.x; i < n; i += kTopkThreads) {
+  for (unsigned i = threadIdx.x; i < n; i += NTHR) {
     const unsigned long long x = cbuf[i];
     int r = 0;
 #pragma unroll 8
     for (unsigned j2 = 0; j2 < n; ++j2) r += cbuf[j2] > x ? 1 : 0;
     if (r < k) sel[r] = x;
   }
-  for (int r = static_cast<int>(n) + threadIdx.x; r < k; r += kTopkThreads) sel[r] = 0ull;
+  for (int r = static_cast<int>(n) + threadIdx.x; r < k; r += NTHR) sel[r] = 0ull;
   __syncthreads();
 }
 
+template <int NTHR = kTopkThreads>
 __device__ __forceinline__ void write_topk(const unsigned long long *sel, int k, int32_t *ids,
                                            float *scores) {
-  for (int r = threadIdx.x; r < k; r += kTopkThreads) {
+  for (int r = threadIdx.x; r < k; r += NTHR) {
     const unsigned long long key = sel[r];
     ids[r] = key ? topk_key_id(key) : -1;
     scores[r] = key ? topk_key_score(key) : -INFINITY;
@@ -207,21 +212,23 @@ __device__ __forceinline__ void write_topk(const unsigned long long *sel, int k,
 // grid (n_split, B).  Warp w of split s holds documents s*kTopkSlice + w*512 ..
 // + 511 (lane l: four runs of 4 from 4 l when the row can be read as float4,
 // else l + 32 j).  With n_split == 1 the result goes straight to ids/scores.
-template <int KL>
-__global__ void __launch_bounds__(kTopkThreads)
+// NTHR threads per CTA (a slice of NTHR x kTopkPerThread documents): 128 for a
+// memory of at most 2,048 documents, so no warp joins the barriers empty-handed.
+template <int KL, int NTHR = kTopkThreads>
+__global__ void __launch_bounds__(NTHR)
 topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__ exclude,
                     int n_docs, int k, int n_split, unsigned long long *__restrict__ cand,
                     int32_t *__restrict__ ids, float *__restrict__ scores) {
-  __shared__ unsigned long long wc[kTopkWarps * KL];
+  __shared__ unsigned long long wc[(NTHR / 32) * KL];
   __shared__ unsigned long long sel[kMaxTopK];
-  __shared__ unsigned long long wt[kTopkWarps + 1], cbuf[kTopkCandCap];
+  __shared__ unsigned long long wt[NTHR / 32 + 1], cbuf[kTopkCandCap];
   const int b = blockIdx.y, split = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(b) * n_docs;
   griddep_wait();
   griddep_launch();
   unsigned long long key[kTopkPerThread];
-  const int dw = split * kTopkSlice + warp * (32 * kTopkPerThread);
+  const int dw = split * (NTHR * kTopkPerThread) + warp * (32 * kTopkPerThread);
   if (exclude == nullptr && (n_docs & 3) == 0 && (reinterpret_cast<uintptr_t>(state) & 15) == 0) {
     // four 16-byte loads per thread: lane takes documents dw + 128 j4 + 4 lane + 0..3
     // (n_docs % 4 == 0, so a vector is either wholly inside the row or wholly past it)
@@ -250,12 +257,13 @@ topk_partial_kernel(const float *__restrict__ state, const uint8_t *__restrict__
       key[j] = ok ? topk_key(state[row + d], d) : 0ull;
     }
   }
-  block_select_topk_fast<KL>(key, k, wc, sel, wt, cbuf);
+  block_select_topk_fast<KL, NTHR>(key, k, wc, sel, wt, cbuf);
   if (n_split == 1) {
-    write_topk(sel, k, ids + static_cast<int64_t>(b) * k, scores + static_cast<int64_t>(b) * k);
+    write_topk<NTHR>(sel, k, ids + static_cast<int64_t>(b) * k,
+                     scores + static_cast<int64_t>(b) * k);
   } else {
     unsigned long long *dst = cand + (static_cast<int64_t>(b) * n_split + split) * k;
-    for (int r = threadIdx.x; r < k; r += kTopkThreads) dst[r] = sel[r];
+    for (int r = threadIdx.x; r < k; r += NTHR) dst[r] = sel[r];
   }
 }
 
