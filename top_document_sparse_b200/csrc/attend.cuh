@@ -7,16 +7,21 @@
 // Kernels:
 //   append_kernel         rotate the new K rows, write K/V into the local cache
 //   attend_simt_kernel    fp32 path (CUDA cores, one warp per query head)
-//   attend_mma_kernel     bf16 path: per (query, kv head, token, context
-//                         split) CTA, 3 warps stream 16-row context blocks
-//                         (cp.async, double-buffered, XOR-swizzled smem) and
-//                         run S^T = K Q^T and O^T += V^T P^T on mma.sync with
-//                         an online softmax (context rows / head dim on M, the
-//                         GQA group's heads on N)
+//   attend_mma_kernel     bf16 one-token (decode) path: per (query, kv head,
+//                         context split) CTA, 3 warps stream 16-row context
+//                         blocks (cp.async, double-buffered, XOR-swizzled
+//                         smem) and run S^T = K Q^T and O^T += V^T P^T on
+//                         mma.sync with an online softmax (context rows / head
+//                         dim on M, the GQA group's heads on N)
 //   attend_combine_kernel merge context splits (log-sum-exp) and advance
 //                         cache_len (a one-split decode call advances it in
 //                         the attention kernel, whose CTAs of one query form
 //                         a cluster)
+//   attend_prefill_kernel bf16 calls of more than one token: per (query, kv
+//                         head, tile of 64 / G tokens) CTA, the tile's query
+//                         rows on M and each staged context block shared by
+//                         its four warps (see below)
+//   advance_kernel        cache_len += tokens where no kernel above does it
 // For a one-token call (decode) the attention kernel appends the new row
 // itself; longer calls run append_kernel first.
 #pragma once

@@ -4,8 +4,10 @@
 // id).  Each (score, id) pair is packed into one order-preserving 64-bit key,
 // so the top-k is a selection of the k largest keys -- exact and
 // deterministic.  Phase 1: one CTA per (query, 4096-document slice) selects
-// its slice's k largest keys; phase 2 merges the slices' candidates.  Both
-// filter first (block_select_topk_fast) and sort only the few survivors.
+// its slice's k largest keys (a memory of at most 2,048 documents: one
+// 128-thread CTA per query, no phase 2); phase 2 merges the slices'
+// candidates.  Both filter first (block_select_topk_fast) and sort only the
+// few survivors.
 #pragma once
 #include "common.cuh"
 #include "ptx.cuh"
