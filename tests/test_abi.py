@@ -89,3 +89,22 @@ def test_calls_reject_null_handles():
     assert lib.msa_step(None, None, None, None, None, None, None, None, None, None) == 1
     assert lib.msa_route_workspace_size(None, 1, 1, 1) == 0
     assert lib.msa_device_error(None, None) == 1
+
+
+def test_adaptive_interleave_validates_before_touching_the_gpu():
+    """msa_interleave_adaptive rejects a null n_rounds and a NaN stop score (INVALID_ARG, with a
+    message) before any CUDA call, so these checks run on a machine without a GPU."""
+    import ctypes
+    lib = msa.lib()
+    n = ctypes.c_int32(0)
+    assert lib.msa_interleave_adaptive(None, None, None, 1, 1, 1, 1, 0.5, None, None, None, None,
+                                       None, None, 0, None) == 1
+    assert b"n_rounds" in lib.msa_last_error()
+    assert lib.msa_interleave_adaptive(None, None, None, 1, 1, 1, 1, float("nan"), None, None,
+                                       None, None, ctypes.addressof(n), None, 0, None) == 1
+    assert b"NaN" in lib.msa_last_error()
+    assert lib.msa_interleave_adaptive(None, None, None, 1, 1, 1, 1, float("-inf"), None, None,
+                                       None, None, ctypes.addressof(n), None, 0, None) == 1
+    assert b"null" in lib.msa_last_error()
+    assert lib.msa_interleave(None, None, None, 1, 1, 1, 1, None, None, None, None, None, 0,
+                              None) == 1
