@@ -421,6 +421,11 @@ def test_interleave_pads_with_minus_one_once_every_document_is_in_the_context():
     ids = [int(r[0][0, 0]) for r in out]
     assert sorted(ids[:4]) == [0, 1, 2, 3] and ids[4:] == [-1, -1]
     assert all(np.isneginf(r[1][0, 0]) for r in out[4:])
+    # rounds 1-4 route the rows of the documents taken in rounds 0-3; round 5 has no rows, so the
+    # final state is the max of the query's and those four documents' cosines: every document
+    # matches its own row exactly, so the state is 1 everywhere
+    _, state, _ = oracle.interleave(Qr, Krb, off, k=1, rounds=6, stop_score=-np.inf)
+    np.testing.assert_allclose(state[0], np.ones(4), atol=1e-12)
 
 
 # ----------------------------------------------------------------------------- golden example
