@@ -106,3 +106,33 @@ def _failing_pins(so_path):
 def test_pins_catch_planted_mistake(workdir, name, edits):
     failed = _failing_pins(_build_mutant(workdir, name, edits))
     assert failed, f"no pin caught the planted mistake {name}"
+
+
+# Mistakes planted in the oracle's Python interleave (the adaptive stop rule and the exclusion
+# padding live there, out of reach of the C mutants above).
+PY_MUTANTS = [
+    ("stop_on_equal_score", "active &= top[:, 0] >= stop_score",
+     "active &= top[:, 0] > stop_score"),
+    ("stopped_round_kept", "ids[~active] = -1", "pass"),
+    ("rounds_counted_for_stopped_queries", "n_rounds += active", "n_rounds += 1"),
+    ("taken_documents_listed_again", "ids[excluded] = -1", "pass"),
+]
+PY_PINS = [getattr(pins, n) for n in sorted(dir(pins))
+           if n.startswith("test_") and ("interleave" in n)]
+
+
+@pytest.mark.parametrize("name,old,new", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_pins_catch_planted_mistake_in_the_interleave(name, old, new, monkeypatch):
+    import inspect
+    src = inspect.getsource(oracle.interleave)
+    assert src.count(old) == 1, f"{name}: pattern must occur once"
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), f"<mutant {name}>", "exec"), ns)
+    monkeypatch.setattr(oracle, "interleave", ns["interleave"])
+    failed = []
+    for pin in PY_PINS:
+        try:
+            pin()
+        except Exception:
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught the planted mistake {name}"

@@ -403,6 +403,12 @@ def test_adaptive_interleave_stop_rule_on_a_hand_worked_chain():
     np.testing.assert_allclose(state[0], [1.0, 0.6, 0.0, -1.0], atol=1e-12)  # D1's row unrouted
 
 
+def test_adaptive_interleave_keeps_a_round_whose_best_score_equals_the_threshold():
+    Qr, Krb, off = _adaptive_docs()                     # round 1's best is exactly 0.6
+    _, _, n = oracle.interleave(Qr, Krb, off, k=1, rounds=3, stop_score=0.6)
+    assert n.tolist() == [3]                            # "below" stops; equal does not
+
+
 def test_adaptive_interleave_limits_reduce_to_fixed_rounds_and_to_round_zero():
     Qr, Krb, off = _adaptive_docs()
     fixed = oracle.interleave(Qr, Krb, off, k=2, rounds=3)
