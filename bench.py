@@ -170,6 +170,8 @@ def build_layers(w, n_layers, seed, msa, t_enc):
     layers = []
     block_docs = max(1, (1 << 18) // max(1, int(off[1] - off[0])))  # ~256K tokens per block
     enc_bytes = 0
+    # every layer's cache length in one tensor, so that one copy sets a decode position
+    lens_all = torch.zeros(n_layers, B, dtype=torch.int32, device=dev)
     for l in range(n_layers):
         L = LayerState()
         L.rk = mem.new_router_keys()
@@ -193,12 +195,12 @@ def build_layers(w, n_layers, seed, msa, t_enc):
             t_enc.append((e0, e1))
             enc_bytes += (K.numel() + V.numel() + Kr.numel()) * K.element_size()
             del K, V, Kr
-        L.dec = msa.LayerDecode(mem, B, k, H_q, cap)
+        L.dec = msa.LayerDecode(mem, B, k, H_q, cap, cache_len=lens_all[l])
         L.Qr_pre = Qr
         L.prefill = (Q, Kn, Vn)
         L.plants = plants
         layers.append(L)
-    return mem, off, layers, enc_bytes
+    return mem, off, layers, enc_bytes, lens_all
 
 
 def prefill(mem, w, layers, msa):
@@ -220,7 +222,6 @@ def prefill(mem, w, layers, msa):
     torch.cuda.synchronize()
     for L in layers:
         L.state0 = L.dec.state.clone()
-        L.len0 = L.dec.cache_len.clone()
         del L.prefill, L.Qr_pre
     return ev
 
@@ -234,8 +235,9 @@ def run_gpu(args, w, world, rank, local):
     es = 2 if w.dtype == "bf16" else 4
     seed = 1234 + rank
     t_enc = []
-    mem, off, layers, enc_bytes = build_layers(w, n_layers, seed, msa, t_enc)
+    mem, off, layers, enc_bytes, lens_all = build_layers(w, n_layers, seed, msa, t_enc)
     pre_ev = prefill(mem, w, layers, msa)
+    len0_all = lens_all.clone()
     enc_ms = sum(a.elapsed_time(b) for a, b in t_enc)
     pre_route_ms = sum(a.elapsed_time(b) for a, b, _ in pre_ev)
     pre_attn_ms = sum(b.elapsed_time(c) for _, b, c in pre_ev)
@@ -257,20 +259,31 @@ def run_gpu(args, w, world, rank, local):
     def reset():
         for L in layers:
             L.dec.state.copy_(L.state0)
-            L.dec.cache_len.copy_(L.len0)
+        lens_all.copy_(len0_all)
+
+    # Decode position s of the episode: every layer's local cache holds T + s rows.  Each
+    # position's step sets that length (one 4 * layers * batch byte copy) before its layers, so a
+    # timed step can run any position and the timed steps can cover the episode uniformly,
+    # whatever --steps is.  (The running routing state is not rewound: it only changes which
+    # documents are retrieved -- the planted ones either way -- not the work.)
+    pos_lens = torch.stack([len0_all + s for s in range(S)])
 
     def step(s, flds, o):
-        if s == 0:
-            reset()
+        lens_all.copy_(pos_lens[s])
         for l, L in enumerate(layers):
             Qr, Q, Kt, Vt = flds[l][s]
             mem.step(L.rk, L.ct, L.dec, Qr, Q, Kt, Vt, o[l])
+
+    def positions(n):
+        """n decode positions spread uniformly over the episode."""
+        return [(i * S) // n for i in range(n)]
 
     # CUDA graphs: one per decode position (inputs differ per position)
     stream = torch.cuda.Stream()
     graphs = []
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
+        reset()
         for s in range(S):  # eager warm pass through every position (also checks the calls)
             step(s, fields, out)
     torch.cuda.synchronize()
@@ -286,8 +299,9 @@ def run_gpu(args, w, world, rank, local):
     torch.cuda.synchronize()
 
     K, Wm = args.steps, args.warmup
-    for i in range(Wm):
-        graphs[i % S].replay()
+    timed_pos = positions(K)
+    for p in positions(max(Wm, 1))[:Wm]:
+        graphs[p].replay()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
@@ -295,8 +309,8 @@ def run_gpu(args, w, world, rank, local):
     with ClockSampler(local) as clk:
         cur = torch.cuda.current_stream()
         e0.record(cur)
-        for i in range(Wm, Wm + K):
-            graphs[i % S].replay()
+        for p in timed_pos:
+            graphs[p].replay()
         e1.record(cur)
         torch.cuda.synchronize()
     barrier(world)
@@ -321,33 +335,30 @@ def run_gpu(args, w, world, rank, local):
         ids_host = [torch.empty(n_layers, B, k, dtype=torch.int32, pin_memory=True)
                     for _ in range(2)]
 
-        def e2e_graph_step(s0, p):
-            if s0 == 0:
-                reset()
+        def e2e_body(p):
             for l, L in enumerate(layers):
                 Qr, Q, Kt, Vt = (d[l] for d in dev_in[p])
                 mem.step(L.rk, L.ct, L.dec, Qr, Q, Kt, Vt, dev_out[p][l])
                 dev_ids[p][l].copy_(L.dec.ids)
 
         g_e2e = {}
-        for s0 in (0, 1):
-            for p in (0, 1):
-                gph = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(gph, stream=stream):
-                    e2e_graph_step(s0, p)
-                g_e2e[(s0, p)] = gph
+        for p in (0, 1):
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph, stream=stream):
+                e2e_body(p)
+            g_e2e[p] = gph
         torch.cuda.synchronize()
         h2d = sum(h[0].numel() * h[0].element_size() for h in hosts)
         d2h = out.numel() * out.element_size() + dev_ids[0].numel() * 4
-        K2 = min(K, 4 * S)
+        K2 = K
         cur = torch.cuda.current_stream()
         s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
         done_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer p copied
         done_comp = [torch.cuda.Event() for _ in range(2)]  # step on buffer p computed
         done_out = [torch.cuda.Event() for _ in range(2)]   # outputs of buffer p copied back
 
-        def copy_in(i):
-            p, s = i % 2, i % S
+        def copy_in(i, s):
+            p = i % 2
             with torch.cuda.stream(s_in):
                 if i >= 2:
                     s_in.wait_event(done_comp[p])           # step i-2 has read buffer p
@@ -355,17 +366,21 @@ def run_gpu(args, w, world, rank, local):
                     d.copy_(h[s], non_blocking=True)
                 done_in[p].record(s_in)
 
-        def run(n):
-            # an episode starts at position 0 (the graph for position 0 resets the state)
-            copy_in(0)
+        def run(pos, graphed):
+            copy_in(0, pos[0])
+            n = len(pos)
             for j in range(n):
                 p = j % 2
                 if j + 1 < n:
-                    copy_in(j + 1)
+                    copy_in(j + 1, pos[j + 1])
                 cur.wait_event(done_in[p])
                 if j >= 2:
                     cur.wait_event(done_out[p])             # step j-2's outputs are on the host
-                g_e2e[(0 if j % S == 0 else 1, p)].replay()
+                lens_all.copy_(pos_lens[pos[j]])            # this step's decode position
+                if graphed:
+                    g_e2e[p].replay()
+                else:
+                    e2e_body(p)
                 done_comp[p].record(cur)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(done_comp[p])
@@ -374,21 +389,30 @@ def run_gpu(args, w, world, rank, local):
                     done_out[p].record(s_out)
             cur.wait_event(done_out[(n - 1) % 2])
 
-        run(min(Wm, S))
-        torch.cuda.synchronize()
-        barrier(world)
-        torch.cuda.synchronize()
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(cur)
-        run(K2)
-        a1.record(cur)
-        torch.cuda.synchronize()
-        barrier(world)
-        ms2 = max_over_ranks(a0.elapsed_time(a1), world)
+        def timed_run(graphed):
+            run(positions(max(Wm, 1)), graphed)
+            torch.cuda.synchronize()
+            barrier(world)
+            torch.cuda.synchronize()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(cur)
+            run(positions(K2), graphed)
+            a1.record(cur)
+            torch.cuda.synchronize()
+            barrier(world)
+            return max_over_ranks(a0.elapsed_time(a1), world)
+
+        ms2 = timed_run(True)
+        ms3 = timed_run(False)
+        assert msa.device_error() == 0
         e2e = {"value": round(world * K2 / (ms2 / 1e3), 2), "unit": "steps/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "tokens_per_s": round(world * K2 * B / (ms2 / 1e3), 1),
-               "pipelined": "inputs of step i+1 and outputs of step i-1 copied while step i runs"}
+               "pipelined": "inputs of step i+1 and outputs of step i-1 copied while step i runs; "
+                            "each step a replayed CUDA graph of its msa_step calls",
+               "eager": {"value": round(world * K2 / (ms3 / 1e3), 2), "unit": "steps/s",
+                         "note": "the same loop with every msa_step called through the C ABI "
+                                 "each step (host validation and launches in the timed region)"}}
         del hosts, dev_in, dev_out, g_e2e
     # ---------------------------------------------------------------- per-kernel timing
     # Route and attention called separately (what msa_step does inside), captured in graphs
@@ -429,7 +453,10 @@ def run_gpu(args, w, world, rank, local):
     route_gbs = route_bytes / (statistics.mean(route_ms) * 1e-3) / 1e9
     attn_bytes = [B * H_kv * (n_mem_rows + c) * 2 * D * es + 2 * B * H_q * D * es for c in attn_ctx]
     attn_gbs = statistics.mean(b / (t * 1e-3) / 1e9 for b, t in zip(attn_bytes, attn_ms))
-    step_bytes = n_layers * (route_bytes + statistics.mean(attn_bytes))
+    # the step's algorithmic bytes at the decode positions the timed steps ran
+    timed_attn_bytes = statistics.mean(B * H_kv * (n_mem_rows + w.query_tokens + p + 1) * 2 * D * es
+                                       + 2 * B * H_q * D * es for p in timed_pos)
+    step_bytes = n_layers * (route_bytes + timed_attn_bytes)
     kernels = {
         "route": {"ms_per_call": round(statistics.mean(route_ms), 5),
                   "bytes_per_call": int(route_bytes), "achieved_gbs": round(route_gbs, 1),
@@ -463,6 +490,8 @@ def run_gpu(args, w, world, rank, local):
                    "query_tokens": w.query_tokens, "decode_positions": S,
                    "heads": f"{H_q}q/{H_kv}kv x {D}, router {w.n_router_heads}x{w.router_dim}",
                    "parallelism": f"replicas x{world}",
+                   "timed_positions": f"{K} steps at decode positions i*{S}//{K}, i < {K} "
+                                      f"(uniform over the {S}-position episode)",
                    "l2": "no flush: every step streams ~%.1f GB > 126 MB L2" % (step_bytes / 1e9),
                    "cuda_graphs": True},
         "tokens_per_s": round(world * K * B / (ms / 1e3), 1),
@@ -480,7 +509,7 @@ def run_gpu(args, w, world, rank, local):
         "e2e": e2e,
     }
     # library kernels in the timed region: the replayed graphs' captured launches
-    res["gpu_launches"] = sum(graph_launches[i % S] for i in range(Wm, Wm + K))
+    res["gpu_launches"] = sum(graph_launches[p] for p in timed_pos)
     return res
 
 
@@ -712,87 +741,150 @@ def run_interleave(w, msa, seed=777, reps=3):
 
 
 # ---------------------------------------------------------------------------- CPU baseline
-class OracleSample:
-    """The fp64 oracle on a bounded sample of the workload's decode step: one decode token for a
-    few queries of one layer, routed against a slice of the documents, top-k over all documents,
-    attention over k retrieved documents plus the local rows.  ``step()`` times one sampled step
-    and extrapolates it linearly to the whole step (every query, layer and document)."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
-    def __init__(self, w, seed, n_docs_sample, queries):
+
+class OracleStep:
+    """The fp64 oracle running whole decode steps of a workload: for every routed layer, route
+    the new token of every query against every document (running max), take the top-k over
+    all documents, and attend over the retrieved documents plus the local rows -- the same work
+    as one GPU step, nothing extrapolated.  Only the memory's values are cheaper to make: a
+    block of documents is encoded by the oracle and repeated to fill the memory (the oracle's
+    cost does not depend on the values), and every layer reads that one memory with its own
+    query tokens and running state."""
+
+    def __init__(self, w, seed, enc_docs=32):
         import oracle
         self.oracle, self.w = oracle, w
         off_full = inputs.doc_offsets(w, seed)
         self.n_docs = off_full.size - 1
-        self.nd = nd = min(n_docs_sample, self.n_docs)
+        nd = min(enc_docs, self.n_docs)
+        assert self.n_docs % nd == 0 and w.doc_len, "fixed-length documents"
         off = off_full[:nd + 1]
-        self.B, T = queries, w.query_tokens
         K, V, Kr = inputs.raw_memory(w, int(off[-1]), seed, "cpu")
-        self.Qr, self.Q, self.Kn, self.Vn = inputs.queries(w, self.B, T + 1, seed + 1, "cpu")
-        self.cho = oracle.doc_chunks(off, w.chunk_len)
-        self.Kb, self.Vb, self.Krb = oracle.encode(K, V, Kr, off, w.chunk_len, w.rope_theta)
-        self.state = oracle.route(self.Qr[:, :T], self.Krb, self.cho)
-        rng = np.random.default_rng(0)
-        self.full_state = np.concatenate(
-            [self.state, rng.uniform(-0.2, 0.2, size=(self.B, self.n_docs - nd))], axis=1)
-        kk = min(w.top_k, nd)
-        self.ids = np.stack([rng.choice(nd, size=kk, replace=False)
-                             for _ in range(self.B)]).astype(np.int32)
+        Kb, Vb, Krb = oracle.encode(K, V, Kr, off, w.chunk_len, w.rope_theta)
+        rep = self.n_docs // nd
+        self.Kb = np.ascontiguousarray(np.tile(Kb, (rep, 1, 1)))
+        self.Vb = np.ascontiguousarray(np.tile(Vb, (rep, 1, 1)))
+        self.Krb = np.ascontiguousarray(np.tile(Krb, (rep, 1, 1)))
+        self.cho = oracle.doc_chunks(off_full, w.chunk_len)
+        B, T, S, L = w.batch, w.query_tokens, w.decode_steps, w.n_layers
+        Qr, Q, Kn, Vn = inputs.queries(w, B, T + S, seed + 1, "cpu")
+        self.Qr, self.Q = Qr, Q
+        self.Kn, self.Vn = oracle.f64(Kn), oracle.f64(Vn)  # converted once, read by every call
+        rng = np.random.default_rng(seed)
+        self.state = [rng.uniform(-0.2, 0.2, size=(B, self.n_docs)) for _ in range(L)]
         self.cores = len(os.sched_getaffinity(0))
 
-    def step(self):
-        o, w, T = self.oracle, self.w, self.w.query_tokens
+    def step(self, p: int) -> float:
+        """Wall seconds of decode step p (local cache of T + p rows before the new token)."""
+        o, w, t = self.oracle, self.w, self.w.query_tokens + p
         t0 = time.perf_counter()
-        o.route(self.Qr[:, T], self.Krb, self.cho, self.state)
-        t1 = time.perf_counter()
-        o.topk(self.full_state, w.top_k)
-        t2 = time.perf_counter()
-        o.attend(self.Q[:, T:T + 1], self.Kn, self.Vn, T, self.Kb, self.Vb, self.cho, self.ids,
-                 w.top_k, w.rope_theta)
-        t3 = time.perf_counter()
-        per_q = ((t1 - t0) * (self.n_docs / self.nd) + (t2 - t1) + (t3 - t2)) / self.B
-        return per_q * w.batch * w.n_layers  # seconds per whole decode step
+        for l in range(w.n_layers):
+            self.state[l] = o.route(self.Qr[:, t], self.Krb, self.cho, self.state[l])
+            ids, _ = o.topk(self.state[l], w.top_k)
+            o.attend(self.Q[:, t:t + 1], self.Kn, self.Vn, t, self.Kb, self.Vb, self.cho, ids,
+                     w.top_k, w.rope_theta)
+        return time.perf_counter() - t0
 
-    def describe(self, reps):
+    def describe(self, n):
         w = self.w
-        return (f"{reps} sampled decode tokens, each for {self.B} queries of one layer: route "
-                f"against {self.nd} of {self.n_docs} documents, top-{w.top_k} over all "
-                f"{self.n_docs}, attention over {w.top_k} docs + {w.query_tokens + 1} local rows; "
-                f"scaled linearly to {w.batch} queries x {w.n_layers} layers x {self.n_docs} "
-                f"documents (extrapolated)")
+        return (f"{n} whole decode steps of {w.name} (every layer of {w.n_layers}, every query "
+                f"of {w.batch}, every document of {self.n_docs}: route, top-{w.top_k}, "
+                f"attention), at decode positions spread over the episode; nothing "
+                f"extrapolated")
 
 
-def cpu_baseline(w, seed=1234, budget_s=12.0):
-    t_start = time.perf_counter()
-    smp = OracleSample(w, seed, n_docs_sample=128, queries=2)
-    times = []
+def oracle_full_configs(seed=1234):
+    """The oracle over the two small workloads in full: the tiny fp32 check (encode, route the
+    query block, top-k, attend) and the 16K-token workload (encode, prefill, then all 64 decode
+    steps), seconds on this host."""
+    import oracle
+    from top_document_sparse_b200.workloads import WORKLOADS as W
+    out = {}
+    w = W["tiny_f32"]
     t0 = time.perf_counter()
-    while not times or time.perf_counter() - t0 < budget_s:
-        times.append(smp.step())
-    step_s = statistics.median(times)
+    off = inputs.doc_offsets(w, seed)
+    K, V, Kr = inputs.raw_memory(w, int(off[-1]), seed, "cpu")
+    Qr, Q, Kn, Vn = inputs.queries(w, w.batch, w.query_tokens, seed + 1, "cpu")
+    t1 = time.perf_counter()
+    Kb, Vb, Krb = oracle.encode(K, V, Kr, off, w.chunk_len, w.rope_theta)
+    cho = oracle.doc_chunks(off, w.chunk_len)
+    st = oracle.route(Qr, Krb, cho)
+    ids, _ = oracle.topk(st, w.top_k)
+    oracle.attend(Q, Kn, Vn, 0, Kb, Vb, cho, ids, w.top_k, w.rope_theta)
+    t2 = time.perf_counter()
+    out["tiny_f32"] = {"pipeline_s": round(t2 - t1, 4), "inputs_s": round(t1 - t0, 3),
+                       "what": "encode 64 docs x 512 tokens, route 4 x 32 tokens, top-4, attend"}
+    w = W["mem16k_bf16"]
+    off = inputs.doc_offsets(w, seed)
+    K, V, Kr = inputs.raw_memory(w, int(off[-1]), seed, "cpu")
+    T, S = w.query_tokens, w.decode_steps
+    Qr, Q, Kn, Vn = inputs.queries(w, w.batch, T + S, seed + 1, "cpu")
+    t0 = time.perf_counter()
+    Kb, Vb, Krb = oracle.encode(K, V, Kr, off, w.chunk_len, w.rope_theta)
+    cho = oracle.doc_chunks(off, w.chunk_len)
+    t1 = time.perf_counter()
+    st = oracle.route(Qr[:, :T], Krb, cho)
+    ids, _ = oracle.topk(st, w.top_k)
+    oracle.attend(Q[:, :T], Kn, Vn, 0, Kb, Vb, cho, ids, w.top_k, w.rope_theta)
+    t2 = time.perf_counter()
+    for s in range(S):
+        st, ids, _, _ = oracle.decode_step(st, Qr[:, T + s], Q[:, T + s], Kn, Vn, T + s, Krb, Kb,
+                                           Vb, cho, w.top_k, w.top_k, w.rope_theta)
+    t3 = time.perf_counter()
+    out["mem16k_bf16"] = {"encode_s": round(t1 - t0, 3), "prefill_s": round(t2 - t1, 3),
+                          "decode_steps": S, "decode_s": round(t3 - t2, 3),
+                          "decode_steps_per_s": round(S / (t3 - t2), 2)}
+    return out
+
+
+def cpu_baseline(w, seed=1234, n_steps=2):
+    t_start = time.perf_counter()
+    smp = OracleStep(w, seed)
+    S = w.decode_steps
+    times = [smp.step((2 * i + 1) * S // (2 * n_steps)) for i in range(n_steps)]
+    step_s = statistics.mean(times)
+    full = oracle_full_configs(seed)
     return {"value": round(1.0 / step_s, 6), "unit": "steps/s", "cores": smp.cores,
-            "kind": "oracle", "sample": smp.describe(len(times)),
+            "cpu_model": cpu_model(), "kind": "oracle", "sample": smp.describe(len(times)),
+            "step_s": [round(t, 3) for t in times],
+            "full_configs": full,
             "seconds": round(time.perf_counter() - t_start, 1)}
 
 
-def run_reference(args, w):
+def run_reference(args, w, budget_s=150.0):
+    """The reference arm: the oracle's whole decode steps (OracleStep), as many of the K asked
+    for as fit in the time budget, at decode positions spread over the episode."""
     K, Wm = args.steps, args.warmup
-    smp = OracleSample(w, 1234, n_docs_sample=32, queries=1)
-    vals = []
+    smp = OracleStep(w, 1234)
+    S = w.decode_steps
     t_all = time.perf_counter()
-    for i in range(Wm + K):
-        v = smp.step()
-        if i >= Wm:
-            vals.append(v)
-        if time.perf_counter() - t_all > 240:
+    if Wm > 0:
+        smp.step(0)
+    vals = []
+    for i in range(K):
+        vals.append(smp.step((i * S) // K))
+        if time.perf_counter() - t_all > budget_s:
             break
-    value = round(1.0 / statistics.median(vals), 6)
+    step_s = statistics.mean(vals)
+    value = round(1.0 / step_s, 6)
     return {
         "metric": METRIC, "impl": "reference", "value": value,
-        "unit": "steps/s", "n_gpus": 1, "steps": len(vals), "warmup": Wm,
-        "ms_per_step": round(1e3 / value, 3), "higher_is_better": True,
+        "unit": "steps/s", "n_gpus": 1, "steps": len(vals), "warmup": min(Wm, 1),
+        "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "layers": w.n_layers, "batch": w.batch, "top_k": w.top_k},
-        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": smp.cores, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": smp.cores,
+                         "cpu_model": cpu_model(), "kind": "oracle",
                          "sample": smp.describe(len(vals))},
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},

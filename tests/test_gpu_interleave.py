@@ -13,6 +13,55 @@ from helpers import small_workload, to64
 pytestmark = pytest.mark.gpu
 
 
+def _valid_topk(ids_b, ref_b, k, tol, what):
+    """ids_b is a correct top-k of the scores ref_b (-inf = not eligible) up to ties within tol:
+    every document scoring clearly above the k-th best is in it, none clearly below."""
+    order = np.lexsort((np.arange(ref_b.size), -ref_b))
+    kth = ref_b[order[k - 1]]
+    assert len(set(ids_b.tolist())) == k, what
+    assert all(ref_b[d] >= kth - tol for d in ids_b), what
+    assert all(d in ids_b for d in np.nonzero(ref_b > kth + tol)[0]), what
+
+
+def _replay_rounds(Qr, Krb, cho, got, sc, k, R, stop, tol):
+    """The oracle replays adaptive interleave rounds on the GPU's own picks (stage by stage):
+    round r routes the rows the GPU's round r-1 retrieved, over the oracle's running state; the
+    GPU's ids of round r must be a valid top-k of the oracle's state among documents not yet in
+    the context, their scores the oracle's, and the stop decisions the oracle's.  Returns the
+    oracle's final state, rounds kept per query and the ids of every kept round."""
+    Q = to64(Qr)
+    B = Q.shape[0]
+    n_docs = cho.size - 1
+    state = np.full((B, n_docs), -np.inf)
+    taken = np.zeros((B, n_docs), dtype=bool)
+    active = np.ones(B, dtype=bool)
+    n_rounds = np.zeros(B, dtype=np.int64)
+    rows = [Q[b] for b in range(B)]
+    kept = [[] for _ in range(B)]
+    for r in range(R):
+        for b in range(B):
+            if active[b] and rows[b].shape[0] > 0:
+                state[b:b + 1] = oracle.route(rows[b][None], Krb, cho, state[b:b + 1])
+        elig = np.where(taken, -np.inf, state)
+        best = elig.max(axis=1)
+        for b in range(B):
+            if active[b]:
+                assert abs(best[b] - stop) > 2 * tol, f"stop decision too close, query {b}"
+        active &= best >= stop
+        n_rounds += active
+        for b in range(B):
+            if not active[b]:
+                assert np.all(got[r, b] == -1) and np.all(np.isneginf(sc[r, b])), (r, b)
+                rows[b] = np.zeros((0,) + Krb.shape[1:])
+                continue
+            _valid_topk(got[r, b], elig[b], k, tol, f"round {r}, query {b}")
+            assert np.all(np.abs(sc[r, b] - elig[b, got[r, b]]) <= tol), (r, b)
+            kept[b].append(got[r, b].tolist())
+            taken[b, got[r, b]] = True
+            rows[b] = np.concatenate([Krb[cho[d]:cho[d + 1]] for d in got[r, b]], axis=0)
+    return state, n_rounds, kept
+
+
 def _chain_memory(seed, dtype, B, T, n_docs_lognormal, k):
     from top_document_sparse_b200 import msa
     w = small_workload(dtype=dtype, n_docs=0, doc_len=0, lognormal=n_docs_lognormal, batch=B,
@@ -153,13 +202,54 @@ def test_interleave_when_queries_run_out_of_documents():
     assert all(sorted(got[:3, b, 0].tolist()) == [0, 1, 2] for b in range(2))
     assert np.all(taken.cpu().numpy() == 1)
     # the state after the last routed round (round 3 routes round 2's document; round 4 has no
-    # rows) is the oracle's, whatever the order of the picks
-    if np.array_equal(got[:3], np.stack([r[0] for r in ref[:3]])):
-        st, st_ref = to64(state), oracle.route(Qr, Krb, mem.doc_chunk_offsets)
-        for r in range(3):
-            rows = [np.concatenate([Krb[mem.doc_chunk_offsets[d]:mem.doc_chunk_offsets[d + 1]]
-                                    for d in got[r, b]])[None] for b in range(2)]
-            st_ref = np.concatenate([oracle.route(rows[b], Krb, mem.doc_chunk_offsets,
-                                                  st_ref[b:b + 1]) for b in range(2)])
-        assert np.all(np.abs(st - st_ref) <= 2e-3)
+    # rows) is the oracle's route of the GPU's own picks, whatever their order
+    st, st_ref = to64(state), oracle.route(Qr, Krb, mem.doc_chunk_offsets)
+    for r in range(3):
+        rows = [np.concatenate([Krb[mem.doc_chunk_offsets[d]:mem.doc_chunk_offsets[d + 1]]
+                                for d in got[r, b]])[None] for b in range(2)]
+        st_ref = np.concatenate([oracle.route(rows[b], Krb, mem.doc_chunk_offsets,
+                                              st_ref[b:b + 1]) for b in range(2)])
+    assert np.all(np.abs(st - st_ref) <= 2e-3)
+    assert msa.device_error() == 0
+
+
+def test_adaptive_interleave_k4_with_mixed_stops_matches_oracle():
+    """k = 4 and a threshold under which, in the same round, some queries stop and the others go
+    on: the stopped queries route zero padding rows with their state saved and restored, the
+    active ones route their new documents' rows.  The oracle runs on the GPU's stored unit router
+    keys (stage-wise), so ids match exactly; the threshold lies between the per-query best
+    background scores of the round after the chain ends, at least 4 x the score tolerance from
+    every best score of every round."""
+    msa, w, off, Qr, chain, mem, rk, _ = _chain_memory(303, "bf16", B=8, T=12,
+                                                        n_docs_lognormal=(200, 1.0, 64, 900, 40000),
+                                                        k=4)
+    tol, R = 2e-3, 5
+    Krb = to64(rk)
+    cho = mem.doc_chunk_offsets
+    fixed = oracle.interleave(Qr, Krb, cho, k=4, rounds=R)
+    best = np.stack([r[1][:, 0] for r in fixed])            # [round][query]
+    every = np.unique(best[np.isfinite(best)])
+    # candidate thresholds: midpoints between consecutive best scores of rounds 3 and 4 that
+    # split round 3's queries; take the one farthest from every decision value
+    b3 = best[3]
+    bg = np.unique(best[3:][np.isfinite(best[3:])])
+    cands = [(np.min(np.abs(every - m)), m) for m in 0.5 * (bg[1:] + bg[:-1])
+             if np.any(b3 < m) and np.any(b3 > m)]
+    margin, stop = max(cands)
+    assert margin > 4 * tol, "no clear threshold in this memory"
+    ids, scores, state, taken, n = mem.interleave_adaptive(rk, Qr.cuda(), k=4, max_rounds=R,
+                                                           stop_score=stop)
+    torch.cuda.synchronize()
+    got, sc = ids.cpu().numpy(), to64(scores)
+    st_ref, n_ref, kept = _replay_rounds(Qr, Krb, cho, got, sc, 4, R, stop, tol)
+    assert n.cpu().numpy().tolist() == n_ref.tolist()
+    assert 3 in n_ref and np.any(n_ref > 3), "some queries stop after round 2, others go on"
+    st = to64(state)
+    fin = np.isfinite(st_ref)
+    assert np.array_equal(np.isfinite(st), fin)
+    assert np.all(np.abs(st[fin] - st_ref[fin]) <= tol)
+    tk = taken.cpu().numpy().astype(bool)
+    for b in range(8):  # the context holds the documents of every kept round but the last round
+        in_ctx = [d for r in kept[b][:R - 1] for d in r]
+        assert set(np.nonzero(tk[b])[0].tolist()) == set(in_ctx), f"query {b}"
     assert msa.device_error() == 0

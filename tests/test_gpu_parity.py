@@ -153,6 +153,12 @@ def test_incremental_update_of_one_document_equals_full_encode(case):
         assert torch.equal(got, ref)
         assert torch.equal(got[keep], old[keep])
         assert not torch.equal(got[~keep], old[~keep])
+    # the re-encoded rows against the oracle's encoding of the new tokens, at the pooling bound
+    sub = dict(off=np.array([0, t1 - t0]), K=new["K"][t0:t1], V=new["V"][t0:t1],
+               Kr=new["Kr"][t0:t1])
+    ref = oracle.encode(sub["K"], sub["V"], sub["Kr"], sub["off"], w.chunk_len, w.rope_theta)
+    c0, c1 = int(cho[d]), int(cho[d + 1])
+    _check_pool(w, sub, ct[c0:c1], rk[c0:c1], rmean[c0:c1], ref)
 
 
 def _check_topk(ids, scores, state, ref_state, k, tol, eligible=None):
@@ -320,20 +326,24 @@ def _attend_calls_match_oracle(dt, D, H_q, H_kv, Ts, k, batch):
 
 
 def test_decode_steps_match_oracle():
-    """16K-token memory: prefill route + attend of the 128-token query, then routed decode steps
-    through msa_step, each compared with the oracle's decode step.  Every query gets k planted
-    documents here so that the top-k boundary is planted-vs-background and the retrieved set is
-    unique at every step (the workload's own 8 plants leave near-ties at rank k)."""
-    import dataclasses
+    """16K-token workload at its stated configuration (8 planted documents per query, k = 16, a
+    128-token query, then all 64 decode steps at batch 1) through msa_step, stage by stage: at
+    every step the running state is the oracle's route of the new token over the oracle's own
+    running state; the retrieved set is checked by the validity rule for near-ties at rank k
+    (only 8 documents are planted, so ranks 9..16 are background documents whose scores may be
+    within the tolerance of each other); the step's attention output is the oracle's attention
+    over the documents the GPU retrieved."""
     msa = _msa()
-    w = dataclasses.replace(WORKLOADS["mem16k_bf16"], planted_per_query=16)
-    n_steps = 12
+    w = WORKLOADS["mem16k_bf16"]
+    assert (w.planted_per_query, w.top_k, w.decode_steps, w.batch) == (8, 16, 64, 1)
+    n_steps = w.decode_steps
     inp = memory_inputs(w, seed=104)
     mem = _build(w, inp, max_local=w.top_k + w.query_tokens + n_steps + 4)
     rk, ct, _ = _encode(mem, inp)
     Kb, Vb, Krb = oracle.encode(inp["K"], inp["V"], inp["Kr"], inp["off"], w.chunk_len,
                                 w.rope_theta)
     B, T, k, H_q = w.batch, w.query_tokens, w.top_k, w.n_q_heads
+    cho = mem.doc_chunk_offsets
     cap = T + n_steps + 2
     layer = msa.LayerDecode(mem, B, k, H_q, cap)
     # prefill: route the whole query block, attend it
@@ -343,25 +353,37 @@ def test_decode_steps_match_oracle():
     mem.sparse_attend(ct, layer.ids, inp["Q"].cuda(), inp["Kn"].cuda(), inp["Vn"].cuda(),
                       layer.k_cache, layer.v_cache, layer.cache_len, k, O,
                       msa.workspace(mem.attend_workspace_size(B, T, k, H_q)))
-    st = oracle.route(inp["Qr"], Krb, mem.doc_chunk_offsets)
+    torch.cuda.synchronize()
+    st = oracle.route(inp["Qr"], Krb, cho)
+    _check_topk(layer.ids, layer.scores, layer.state, st, k, SCORE_TOL["bf16"])
+    pb, pd, _, _ = inp["plants"]
+    ref, _, _ = oracle.attend(inp["Q"], inp["Kn"], inp["Vn"], 0, Kb, Vb, cho,
+                              layer.ids.cpu().numpy(), k, w.rope_theta)
+    assert_close(O, ref, attn_tol("bf16", ref), "prefill attention output")
     dec = inputs.queries(w, B, n_steps, seed=777)
     Khist = torch.cat([inp["Kn"], dec[2]], dim=1)
     Vhist = torch.cat([inp["Vn"], dec[3]], dim=1)
+    near_ties = 0
     for s in range(n_steps):
         Ot = torch.empty(B, H_q, w.head_dim, dtype=torch.bfloat16, device="cuda")
         mem.step(rk, ct, layer, dec[0][:, s].cuda().contiguous(), dec[1][:, s].cuda().contiguous(),
                  dec[2][:, s].cuda().contiguous(), dec[3][:, s].cuda().contiguous(), Ot)
         torch.cuda.synchronize()
-        st, ids_o, top_o, O_ref = oracle.decode_step(st, dec[0][:, s], dec[1][:, s], Khist, Vhist,
-                                                     T + s, Krb, Kb, Vb, mem.doc_chunk_offsets, k,
-                                                     k, w.rope_theta)
+        st = oracle.route(dec[0][:, s:s + 1], Krb, cho, st)
         assert_close(layer.state, st, SCORE_TOL["bf16"], f"running state, step {s}")
         _check_topk(layer.ids, layer.scores, layer.state, st, k, SCORE_TOL["bf16"])
-        # same set; the rank order among near-equal scores changes only rounding
-        assert set(layer.ids.cpu().numpy()[0].tolist()) == set(ids_o[0].tolist())
-        assert_close(Ot, O_ref, attn_tol("bf16", O_ref), f"decode output, step {s}")
+        ids_gpu = layer.ids.cpu().numpy()
+        ids_o, _ = oracle.topk(st, k)
+        near_ties += int(set(ids_gpu[0].tolist()) != set(ids_o[0].tolist()))
+        for b, d in zip(pb, pd):  # the planted documents stay retrieved
+            assert d in ids_gpu[b], f"planted document {d} lost at step {s}"
+        O_ref, _, rs = oracle.attend(dec[1][:, s:s + 1], Khist, Vhist, T + s, Kb, Vb, cho, ids_gpu,
+                                     k, w.rope_theta)
+        np.testing.assert_allclose(rs, 1.0, atol=1e-12)
+        assert_close(Ot, O_ref[:, 0], attn_tol("bf16", O_ref[:, 0]), f"decode output, step {s}")
     assert layer.cache_len.cpu().tolist() == [T + n_steps]
     assert msa.device_error() == 0
+    print(f"64 decode steps: {near_ties} steps with a different (valid) set at rank k")
 
 
 def test_device_bounds_checks_raise_the_error_word():

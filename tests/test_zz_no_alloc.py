@@ -83,3 +83,37 @@ def test_static_scratch_rejects_calls_beyond_its_size():
     torch.cuda.synchronize()
     assert lens.cpu().tolist() == [0] * B and bool((O == 7.0).all())
     assert msa.device_error() == 0
+
+
+def test_static_scratch_reports_bad_shapes_before_sizing_its_scratch():
+    """The shape checks of every attention call run before the static scratch is sized: a query
+    head count that is not a multiple of the kv heads is an invalid argument (not a scratch size
+    refusal) even when the call's split-context scratch would not fit the array, and nothing is
+    enqueued."""
+    from top_document_sparse_b200 import msa
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    B, k, H_kv, D, cap = 4, 4, 2, 128, 512
+    T = (3 * sms - 1) // (B * H_kv)
+    w = small_workload(n_q_heads=32, n_kv_heads=H_kv, head_dim=D, batch=B, top_k=k,
+                       n_docs=12, doc_len=448)
+    inp = memory_inputs(w, seed=912)
+    mem = msa.Memory(inp["off"], w.chunk_len, H_kv, D, w.n_router_heads, w.router_dim,
+                     torch.bfloat16, w.rope_theta, k + cap)
+    assert mem.attend_workspace_size(B, T, k, 32) > (4 << 20)
+    ct = torch.zeros(mem.n_chunks, 2, H_kv, D, dtype=torch.bfloat16, device="cuda")
+    Kn = torch.zeros(B, T, H_kv, D, dtype=torch.bfloat16, device="cuda")
+    Kc = torch.zeros(B, cap, H_kv, D, dtype=torch.bfloat16, device="cuda")
+    ids = torch.zeros(B, k, dtype=torch.int32, device="cuda")
+    lens = torch.zeros(B, dtype=torch.int32, device="cuda")
+    Q = torch.zeros(B, T, 33, D, dtype=torch.bfloat16, device="cuda")
+    O = torch.full_like(Q, 7.0)
+    for H_q in (33, 0):  # 33 query heads over 2 kv heads; no query head
+        st = msa.lib().msa_sparse_attend_static(
+            mem.handle, ct.data_ptr(), ids.data_ptr(), B, k, T, H_q, Q.data_ptr(), Kn.data_ptr(),
+            Kn.data_ptr(), Kc.data_ptr(), Kc.data_ptr(), lens.data_ptr(), cap, k, O.data_ptr(),
+            torch.cuda.current_stream().cuda_stream)
+        assert st == 1, msa.lib().msa_last_error()
+        assert b"multiple of n_kv_heads" in msa.lib().msa_last_error()
+    torch.cuda.synchronize()
+    assert lens.cpu().tolist() == [0] * B and bool((O == 7.0).all())
+    assert msa.device_error() == 0

@@ -443,11 +443,10 @@ msa_status dispatch_group(int G, const msa_memory *mem, const void *content, con
 #undef MSA_G
 }
 
-msa_status attend_impl(const msa_memory *mem, const void *content, const int32_t *ids,
-                       const int32_t *slots, int slot_chunks, int B, int k, int T, int H_q,
-                       const void *Q, const void *K_new, const void *V_new, void *K_cache,
-                       void *V_cache, int32_t *cache_len, int cap, int pos_offset, void *O,
-                       void *ws, size_t ws_bytes, cudaStream_t st, bool early = false) {
+// Shape checks shared by every attention entry point; they run before any
+// scratch is sized or anything is enqueued.
+msa_status attend_shape_check(const msa_memory *mem, int B, int k, int T, int H_q, int cap,
+                              int pos_offset) {
   if (!mem) return fail(MSA_ERR_INVALID_ARG, "null memory");
   if (B < 1 || T < 1) return fail(MSA_ERR_INVALID_ARG, "batch and tokens must be >= 1");
   if (k < 0 || k > msa::kMaxTopK) return fail(MSA_ERR_INVALID_ARG, "k=%d out of range", k);
@@ -460,17 +459,27 @@ msa_status attend_impl(const msa_memory *mem, const void *content, const int32_t
     return fail(MSA_ERR_INVALID_ARG,
                 "pos_offset=%d + cache_capacity=%d must be <= max_local_position=%d", pos_offset,
                 cap, mem->max_local_position);
+  if (static_cast<int64_t>(k) * mem->max_doc_chunks > msa::kMaxMemRows)
+    return fail(MSA_ERR_UNSUPPORTED, "k * max_doc_chunks = %lld exceeds %d retrieved rows",
+                (long long)k * mem->max_doc_chunks, msa::kMaxMemRows);
+  if (static_cast<int64_t>(B) * T > 2147483647LL / 64)
+    return fail(MSA_ERR_UNSUPPORTED, "batch * tokens too large");
+  return MSA_OK;
+}
+
+msa_status attend_impl(const msa_memory *mem, const void *content, const int32_t *ids,
+                       const int32_t *slots, int slot_chunks, int B, int k, int T, int H_q,
+                       const void *Q, const void *K_new, const void *V_new, void *K_cache,
+                       void *V_cache, int32_t *cache_len, int cap, int pos_offset, void *O,
+                       void *ws, size_t ws_bytes, cudaStream_t st, bool early = false) {
+  const msa_status chk = attend_shape_check(mem, B, k, T, H_q, cap, pos_offset);
+  if (chk != MSA_OK) return chk;
   if (!content || (k > 0 && !ids) || !Q || !K_new || !V_new || !K_cache || !V_cache ||
       !cache_len || !O)
     return fail(MSA_ERR_INVALID_ARG, "null pointer argument");
   if (!aligned16(content) || !aligned16(Q) || !aligned16(K_new) || !aligned16(V_new) ||
       !aligned16(K_cache) || !aligned16(V_cache) || !aligned16(O) || !aligned16(ws))
     return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-  if (static_cast<int64_t>(k) * mem->max_doc_chunks > msa::kMaxMemRows)
-    return fail(MSA_ERR_UNSUPPORTED, "k * max_doc_chunks = %lld exceeds %d retrieved rows",
-                (long long)k * mem->max_doc_chunks, msa::kMaxMemRows);
-  if (static_cast<int64_t>(B) * T > 2147483647LL / 64)
-    return fail(MSA_ERR_UNSUPPORTED, "batch * tokens too large");
   AttendPlan plan = plan_attend(mem, B, T, k, H_q, cap);
   plan.early = early ? 1 : 0;
   if (ws_bytes < plan.bytes || (plan.bytes > 0 && !ws))
@@ -764,10 +773,9 @@ msa_status msa_sparse_attend_static(const msa_memory *mem, const void *content,
                                     const void *V_new, void *K_cache, void *V_cache,
                                     int32_t *cache_len, int32_t cache_capacity,
                                     int32_t pos_offset, void *O, msa_stream stream) {
-  if (!mem) return fail(MSA_ERR_INVALID_ARG, "null memory");
-  if (batch < 1 || tokens < 1 || k < 0 || k > msa::kMaxTopK || n_q_heads < 1 ||
-      cache_capacity < 1)
-    return fail(MSA_ERR_INVALID_ARG, "bad batch, tokens, k, n_q_heads or cache_capacity");
+  const msa_status chk =
+      attend_shape_check(mem, batch, k, tokens, n_q_heads, cache_capacity, pos_offset);
+  if (chk != MSA_OK) return chk;
   const AttendPlan plan = plan_attend(mem, batch, tokens, k, n_q_heads, cache_capacity);
   if (plan.bytes > kStaticAttendScratchBytes)
     return fail(MSA_ERR_UNSUPPORTED,

@@ -362,7 +362,7 @@ class LayerDecode:
     """Per-layer decode buffers (all torch-allocated) bundled as an msa_decode_state."""
 
     def __init__(self, mem: Memory, batch: int, k: int, n_q_heads: int, cache_capacity: int,
-                 pos_offset: int | None = None, device="cuda"):
+                 pos_offset: int | None = None, device="cuda", cache_len=None):
         self.state = torch.full((batch, mem.n_docs), float("-inf"), dtype=torch.float32,
                                 device=device)
         self.ids = torch.zeros(batch, k, dtype=torch.int32, device=device)
@@ -370,7 +370,13 @@ class LayerDecode:
         self.k_cache = torch.zeros(batch, cache_capacity, mem.n_kv_heads, mem.head_dim,
                                    dtype=mem.dtype, device=device)
         self.v_cache = torch.zeros_like(self.k_cache)
-        self.cache_len = torch.zeros(batch, dtype=torch.int32, device=device)
+        # cache_len may be a caller's view (e.g. one row of a [layers][batch] tensor, so that
+        # every layer's length can be set by one copy)
+        if cache_len is None:
+            cache_len = torch.zeros(batch, dtype=torch.int32, device=device)
+        if cache_len.shape != (batch,) or cache_len.dtype != torch.int32:
+            raise ValueError("cache_len must be int32 [batch]")
+        self.cache_len = cache_len
         self.workspace = workspace(mem.step_workspace_size(batch, k, n_q_heads), device)
         self.pos_offset = k if pos_offset is None else pos_offset
         self.c = DecodeState(batch=batch, top_k=k, n_q_heads=n_q_heads,
