@@ -147,9 +147,12 @@ def test_full_size_interleave_on_sampled_queries():
     round, and two that found every hop -- are replayed by the oracle round by round on the GPU's
     stored unit router keys and on the GPU's own picks: each round's ids must be a valid top-k
     of the oracle's state among the documents not yet in the context (ties within the score
-    tolerance allowed), with the oracle's scores.  A hop the GPU missed is then also outside the
-    oracle's top-k for that round: the misses come from the method (a query's retrieved
-    documents can carry it into another query's chain), not from the kernels."""
+    tolerance allowed), with the oracle's scores.  A hop the GPU missed is outside the oracle's
+    top-k of that round too, or ties with its k-th score: a hop scores the designed 0.6 x 0.8 =
+    0.48 against the previous hop's rows, and so do the next hops of the other queries' chains
+    that a round has pulled into this query's context, so up to k documents can sit at 0.48
+    apart only by the rounding of stored keys.  The misses come from the method and the
+    workload, not from the kernels."""
     from top_document_sparse_b200 import msa
     w = WORKLOADS["interleave_bf16"]
     seed = 777
@@ -175,6 +178,7 @@ def test_full_size_interleave_on_sampled_queries():
     cho = mem.doc_chunk_offsets
     Q = to64(Qr)
     tol = 2e-3
+    miss_kinds = []
     for q in sample:
         state = np.full((1, mem.n_docs), -np.inf)
         taken = np.zeros(mem.n_docs, dtype=bool)
@@ -189,8 +193,12 @@ def test_full_size_interleave_on_sampled_queries():
             assert all(elig[d] >= kth - tol for d in g), (q, r)
             assert all(d in g for d in np.nonzero(elig > kth + tol)[0]), (q, r)
             assert np.all(np.abs(sc[r, q] - elig[g]) <= tol), (q, r)
-            if not hit[q, r]:  # the oracle does not retrieve the missed hop either
-                assert elig[chain[q, r]] < kth - tol, (q, r)
+            if not hit[q, r]:  # the oracle leaves the missed hop out too, or it ties at rank k
+                h = chain[q, r]
+                in_oracle = h in order[:k]
+                assert not in_oracle or abs(elig[h] - kth) <= tol, (q, r)
+                miss_kinds.append("tie at rank k" if abs(elig[h] - kth) <= tol else "below")
             taken[g] = True
             rows = np.concatenate([Krb[cho[d]:cho[d + 1]] for d in g], axis=0)
-    print(f"interleave: {len(missed)} of {B} queries missed a hop; sampled {sample}")
+    print(f"interleave: {len(missed)} of {B} queries missed a hop; sampled {sample}; "
+          f"the missed hops against the oracle's k-th score: {miss_kinds}")
