@@ -341,15 +341,21 @@ MSA_API msa_status msa_interleave_adaptive(const msa_memory *mem, const void *ro
  *
  * A fetcher manages a device slot cache for one layer's content:
  *   content_host : PINNED host memory [C][2][H_kv][D] written by
- *                  msa_encode_memory (it may write host memory directly)
+ *                  msa_encode_memory (it may write host memory directly); it
+ *                  must be mapped into the device address space (pinned memory
+ *                  is, on every 64-bit system with unified addressing)
  *   slot_cache   : device memory of n_slots * doc_content_stride bytes
  *                  (msa_memory_get_info), one document per slot
- *   n_slots      : >= max_batch * max_k, so one call's documents always fit
+ *   n_slots      : >= max_batch * max_k, so one call's documents always fit;
+ *                  max_batch * max_k <= 4096
  *   flags        : MSA_FETCH_COLD forgets every resident document at each
  *                  fetch (every selected document crosses the host link)
- * The fetcher allocates small host-side tables, two events, pinned host
- * staging for max_batch * max_k ids, slots and copy-list entries, and device
- * arrays of the same sizes; it does not own content_host or slot_cache.
+ * The fetcher's bookkeeping lives in device memory it allocates (the document
+ * -> slot map and a claim word per document, the slot -> document map and use
+ * stamps per slot, the slot of each (query, rank), the copy list, a small
+ * scratch array), so no fetch
+ * reads anything back to the host; it also creates two events.  It does not
+ * own content_host or slot_cache.  msa_fetcher_destroy frees what it made.
  */
 typedef struct msa_fetcher msa_fetcher;
 #define MSA_FETCH_COLD 0x1u
@@ -358,22 +364,25 @@ MSA_API msa_status msa_fetcher_create(const msa_memory *mem, const void *content
                                       void *slot_cache, int32_t n_slots, int32_t max_batch,
                                       int32_t max_k, uint32_t flags, msa_fetcher **out);
 MSA_API msa_status msa_fetcher_destroy(msa_fetcher *f);
-/* Totals since creation: (query, rank) hits and misses, documents copied,
- * bytes copied over the host link. */
+/* Totals since creation: (query, rank) hits, misses (documents copied),
+ * documents copied, bytes copied over the host link.  Synchronises the device
+ * to read them. */
 MSA_API msa_status msa_fetcher_stats(const msa_fetcher *f, int64_t *hits, int64_t *misses,
                                      int64_t *copies, int64_t *bytes);
 
 /*
- * Make the documents ids[batch][k] (device) resident in the slot cache.
- * Reads the ids back to the host (synchronising `stream` up to that copy),
- * keeps resident documents, chooses victim slots (a clock over the slots not
- * used by this call) for the others and, on `fetch_stream`, uploads the slot
- * of every (query, rank) and copies every missing document's contiguous chunk
- * rows over the host link: one gather kernel reading content_host through its
- * device mapping (one CTA per document), or one cudaMemcpyAsync per document
- * when content_host is not mapped into the device address space.  Then makes
- * `stream` wait for `fetch_stream`.  Ids outside [0, n_docs) get slot 0 and are skipped by the
- * attention (device error word).  fetch_stream may equal stream.
+ * Make the documents ids[batch][k] (device) resident in the slot cache, with
+ * no host round trip: on `stream` (after the kernel that writes ids) one kernel
+ * keeps the resident documents, gives every missing document a victim slot (a
+ * clock over the slots not used by this call; a document wanted by several
+ * (query, rank) entries is copied once, by the lowest entry) and writes the
+ * slot of every (query, rank) and the list of copies; then, on `fetch_stream`,
+ * one gather kernel copies every missing document's contiguous chunk rows from
+ * content_host through its device mapping (one CTA per document) over the host
+ * link.  `stream` then waits for `fetch_stream`.  fetch_stream may equal
+ * stream.  Ids outside [0, n_docs) get slot 0 and are skipped by the attention
+ * (device error word).  Calls of one fetcher must be ordered (they share its
+ * bookkeeping); a whole step can be captured in a CUDA graph.
  */
 MSA_API msa_status msa_fetch(msa_fetcher *f, const int32_t *ids, int32_t batch, int32_t k,
                              msa_stream stream, msa_stream fetch_stream);
@@ -387,14 +396,42 @@ MSA_API msa_status msa_sparse_attend_fetched(
     int32_t pos_offset, void *O, void *workspace, size_t workspace_bytes, msa_stream stream);
 
 /* msa_step with the content in the host tier: route, msa_fetch, then the
- * attention over the fetched rows.  Synchronises `stream` once (the id
- * read-back). */
+ * attention over the fetched rows.  Nothing is read back to the host. */
 MSA_API msa_status msa_step_host(const msa_memory *mem, const void *router_keys, msa_fetcher *f,
                                  const msa_decode_state *st, const void *Qr_tok,
                                  const void *Q_tok, const void *K_tok, const void *V_tok,
                                  void *O_tok, msa_stream stream, msa_stream fetch_stream);
 
-/* Read and clear the device error word of the current device (synchronises
+/*
+ * Memory Parallel [Evermind summary sec. 4B "Memory Parallel & Tiered Storage":
+ * the routing keys are split over GPUs, the query goes to every GPU, each scores
+ * its own part and the results are reduced to one global top-k; b-lab.team item
+ * 2, the inference engine serving 100M tokens on two GPUs].  The memory's
+ * documents are cut into contiguous ranges ("shards"); each shard is an
+ * msa_memory over its range (document 0 of shard s is global document
+ * shard_doc_base[s]) and routes with msa_route as usual, keeping its top k_cand
+ * as (score, shard-local id).  msa_topk_merge merges every shard's candidates
+ * into the global top-k:
+ *   cand_scores, cand_ids : device [n_shards][batch][k_cand], each shard's
+ *                 msa_route output (ids < 0 are padding and are skipped)
+ *   shard_doc_base : HOST array [n_shards], non-decreasing, >= 0
+ *   ids, scores : device [batch][k] out, global document ids by (score
+ *                 descending, global id ascending); padded with -1 / -inf when
+ *                 fewer than k candidates are valid
+ * With k_cand >= k the result is bit-identical to msa_route over the whole
+ * memory: a document's score does not depend on the partition, and the merge
+ * orders (score, global id) exactly as the single-memory top-k does.  The
+ * candidates reach this GPU by any means -- an all-gather of batch * k_cand *
+ * 8 bytes per shard over NCCL, or, for logical shards on one GPU, the shards'
+ * own output buffers.  Errors: INVALID_ARG (bad counts, k > n_shards * k_cand,
+ * bases out of order), UNSUPPORTED (more than 4096 candidates per query), CUDA.
+ */
+MSA_API msa_status msa_topk_merge(const float *cand_scores, const int32_t *cand_ids,
+                                  int32_t n_shards, int32_t batch, int32_t k_cand,
+                                  const int32_t *shard_doc_base, int32_t k, int32_t *ids,
+                                  float *scores, msa_stream stream);
+
+/* Read and clear the device error word of the current device (synchronises/* Read and clear the device error word of the current device (synchronises
  * `stream`).  *bits receives the MSA_DEVERR_* bits; returns MSA_ERR_TIMEOUT or
  * MSA_ERR_STATE when a bit was set, else MSA_OK. */
 MSA_API msa_status msa_device_error(uint32_t *bits, msa_stream stream);

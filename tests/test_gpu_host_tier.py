@@ -113,3 +113,45 @@ def test_fetcher_rejects_bad_arguments():
     f = msa.Fetcher(mem, ct_host, n_slots=6, max_batch=2, max_k=3)
     with pytest.raises(msa.MsaError):
         f.fetch(torch.zeros(3, 3, dtype=torch.int32, device="cuda"))      # batch beyond max
+
+
+def test_host_tier_step_captured_in_a_cuda_graph_equals_eager_steps():
+    """The fetch reads nothing back to the host (slots are assigned on the device), so a whole
+    host-tier decode step -- route, slot assignment, gather over the host link, attention --
+    can be captured in a CUDA graph; replayed step by step it gives exactly the eager steps,
+    which give exactly the device-resident steps.  Few slots, so documents are evicted."""
+    msa, w, inp, mem, rk, ct_dev, ct_host = _setup(204, n_docs=48, doc_len=384, B=2, k=4, T=8)
+    B, k, H_q, D = w.batch, w.top_k, w.n_q_heads, w.head_dim
+    f_e = msa.Fetcher(mem, ct_host, n_slots=B * k + 1, max_batch=B, max_k=k)
+    f_g = msa.Fetcher(mem, ct_host, n_slots=B * k + 1, max_batch=B, max_k=k)
+    lay_d, lay_e, lay_g = (msa.LayerDecode(mem, B, k, H_q, 10) for _ in range(3))
+    fs = torch.cuda.Stream()
+    cur = torch.cuda.Stream()
+    tok = [inp[n][:, 0].cuda().contiguous() for n in ("Qr", "Q", "Kn", "Vn")]  # static inputs
+    Og = torch.empty(B, H_q, D, dtype=torch.bfloat16, device="cuda")
+    with torch.cuda.stream(cur):  # one eager call on this stream first (kernel attributes)
+        f_g.step(rk, lay_g, *tok, Og, fetch_stream=fs)
+    torch.cuda.synchronize()
+    lay_g.state.fill_(float("-inf"))
+    lay_g.cache_len.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cur):
+        f_g.step(rk, lay_g, *tok, Og, fetch_stream=fs)
+    for t in range(8):
+        x = [inp[n][:, t].cuda().contiguous() for n in ("Qr", "Q", "Kn", "Vn")]
+        Od = torch.empty(B, H_q, D, dtype=torch.bfloat16, device="cuda")
+        Oe = torch.empty_like(Od)
+        mem.step(rk, ct_dev, lay_d, *x, Od)
+        f_e.step(rk, lay_e, *x, Oe, fetch_stream=fs)
+        for dst, src in zip(tok, x):
+            dst.copy_(src)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(lay_e.ids, lay_d.ids) and torch.equal(Oe, Od), f"eager, step {t}"
+        assert torch.equal(lay_g.ids, lay_e.ids) and torch.equal(Og, Oe), f"graph, step {t}"
+    assert lay_g.cache_len.cpu().tolist() == [8] * B
+    s_e, s_g = f_e.stats(), f_g.stats()
+    assert s_e["misses"] >= B * k and s_e["hits"] >= 1
+    assert msa.device_error() == 0
+    del g

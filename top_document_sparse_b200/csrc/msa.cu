@@ -825,6 +825,9 @@ msa_status msa_fetcher_create(const msa_memory *mem, const void *content_host, v
   *out = nullptr;
   if (max_batch < 1 || max_k < 1 || max_k > msa::kMaxTopK)
     return fail(MSA_ERR_INVALID_ARG, "max_batch >= 1 and 1 <= max_k <= %d required", msa::kMaxTopK);
+  if (static_cast<int64_t>(max_batch) * max_k > msa::kAssignMaxIds)
+    return fail(MSA_ERR_UNSUPPORTED, "max_batch * max_k = %lld exceeds %d ids per fetch",
+                (long long)max_batch * max_k, msa::kAssignMaxIds);
   if (static_cast<int64_t>(n_slots) < static_cast<int64_t>(max_batch) * max_k)
     return fail(MSA_ERR_INVALID_ARG, "n_slots=%d < max_batch * max_k = %lld", n_slots,
                 (long long)max_batch * max_k);
@@ -835,9 +838,15 @@ msa_status msa_fetcher_create(const msa_memory *mem, const void *content_host, v
     cudaGetLastError();
     return fail(MSA_ERR_INVALID_ARG, "content_host must be pinned (page-locked) host memory");
   }
+  void *dev = nullptr;
+  if (cudaHostGetDevicePointer(&dev, const_cast<void *>(content_host), 0) != cudaSuccess || !dev) {
+    cudaGetLastError();
+    return fail(MSA_ERR_UNSUPPORTED, "content_host is not mapped into the device address space");
+  }
   auto f = new msa_fetcher();
   f->mem = mem;
   f->content_host = static_cast<const uint8_t *>(content_host);
+  f->content_dev = static_cast<const uint8_t *>(dev);
   f->slot_cache = static_cast<uint8_t *>(slot_cache);
   f->n_slots = n_slots;
   f->max_batch = max_batch;
@@ -845,38 +854,41 @@ msa_status msa_fetcher_create(const msa_memory *mem, const void *content_host, v
   f->flags = flags;
   f->row_bytes = static_cast<size_t>(2) * mem->H_kv * mem->D * elem_size(mem->dtype);
   f->slot_bytes = f->row_bytes * mem->max_doc_chunks;
-  f->doc_slot.assign(mem->n_docs, -1);
-  f->slot_doc.assign(n_slots, -1);
-  f->slot_stamp.assign(n_slots, 0);
   const size_t n = static_cast<size_t>(max_batch) * max_k;
-  if (cudaHostAlloc(reinterpret_cast<void **>(&f->h_ids), n * 4, cudaHostAllocDefault) != cudaSuccess ||
-      cudaHostAlloc(reinterpret_cast<void **>(&f->h_slots), n * 4, cudaHostAllocDefault) != cudaSuccess ||
-      cudaMalloc(reinterpret_cast<void **>(&f->d_slots), n * 4) != cudaSuccess ||
-      cudaEventCreateWithFlags(&f->ev_ids, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&f->ev_fetch, cudaEventDisableTiming) != cudaSuccess ||
-      cudaHostAlloc(reinterpret_cast<void **>(&f->h_list), n * 3 * 8, cudaHostAllocDefault) != cudaSuccess ||
-      cudaMalloc(reinterpret_cast<void **>(&f->d_list), n * 3 * 8) != cudaSuccess) {
+  const size_t nd = static_cast<size_t>(mem->n_docs);
+  auto dmalloc = [](void *p, size_t bytes) {
+    return cudaMalloc(reinterpret_cast<void **>(p), bytes) == cudaSuccess;
+  };
+  bool ok = dmalloc(&f->d_doc_slot, nd * 4) && dmalloc(&f->d_claim, nd * 4) &&
+            dmalloc(&f->d_slot_doc, static_cast<size_t>(n_slots) * 4) &&
+            dmalloc(&f->d_slot_stamp, static_cast<size_t>(n_slots) * 4) &&
+            dmalloc(&f->d_ctl, msa::kCtlN * 8) && dmalloc(&f->d_slots, n * 4) &&
+            dmalloc(&f->d_list, n * 3 * 8) && dmalloc(&f->d_scratch, msa::kAssignScratch * 4) &&
+            cudaEventCreateWithFlags(&f->ev_ids, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&f->ev_fetch, cudaEventDisableTiming) == cudaSuccess;
+  // bookkeeping: no document resident, no claim (any value above every index), stamps 0
+  ok = ok && cudaMemset(f->d_doc_slot, 0xFF, nd * 4) == cudaSuccess &&
+       cudaMemset(f->d_claim, 0x7F, nd * 4) == cudaSuccess &&
+       cudaMemset(f->d_slot_doc, 0xFF, static_cast<size_t>(n_slots) * 4) == cudaSuccess &&
+       cudaMemset(f->d_slot_stamp, 0, static_cast<size_t>(n_slots) * 4) == cudaSuccess &&
+       cudaMemset(f->d_ctl, 0, msa::kCtlN * 8) == cudaSuccess &&
+       cudaDeviceSynchronize() == cudaSuccess;
+  if (!ok) {
     cudaGetLastError();
     msa_fetcher_destroy(f);
-    return fail(MSA_ERR_OUT_OF_MEMORY, "could not allocate the fetcher's staging buffers");
+    return fail(MSA_ERR_OUT_OF_MEMORY, "could not allocate the fetcher's bookkeeping");
   }
-  // the gather kernel reads the content through its device mapping when it has one
-  void *dev = nullptr;
-  if (cudaHostGetDevicePointer(&dev, const_cast<void *>(content_host), 0) == cudaSuccess && dev)
-    f->content_dev = static_cast<const uint8_t *>(dev);
-  else
-    cudaGetLastError();
   *out = f;
   return MSA_OK;
 }
 
 msa_status msa_fetcher_destroy(msa_fetcher *f) {
   if (!f) return fail(MSA_ERR_INVALID_ARG, "null fetcher");
-  if (f->h_ids) cudaFreeHost(f->h_ids);
-  if (f->h_slots) cudaFreeHost(f->h_slots);
-  if (f->d_slots) cudaFree(f->d_slots);
-  if (f->h_list) cudaFreeHost(f->h_list);
-  if (f->d_list) cudaFree(f->d_list);
+  for (void *p : {static_cast<void *>(f->d_doc_slot), static_cast<void *>(f->d_claim),
+                  static_cast<void *>(f->d_slot_doc), static_cast<void *>(f->d_slot_stamp),
+                  static_cast<void *>(f->d_ctl), static_cast<void *>(f->d_slots),
+                  static_cast<void *>(f->d_list), static_cast<void *>(f->d_scratch)})
+    if (p) cudaFree(p);
   if (f->ev_ids) cudaEventDestroy(f->ev_ids);
   if (f->ev_fetch) cudaEventDestroy(f->ev_fetch);
   delete f;
@@ -886,10 +898,13 @@ msa_status msa_fetcher_destroy(msa_fetcher *f) {
 msa_status msa_fetcher_stats(const msa_fetcher *f, int64_t *hits, int64_t *misses,
                              int64_t *copies, int64_t *bytes) {
   if (!f) return fail(MSA_ERR_INVALID_ARG, "null fetcher");
-  if (hits) *hits = f->hits;
-  if (misses) *misses = f->misses;
-  if (copies) *copies = f->copies;
-  if (bytes) *bytes = f->bytes;
+  int64_t ctl[msa::kCtlN];
+  MSA_CUDA(cudaDeviceSynchronize());
+  MSA_CUDA(cudaMemcpy(ctl, f->d_ctl, sizeof(ctl), cudaMemcpyDeviceToHost));
+  if (hits) *hits = ctl[msa::kCtlHits];
+  if (misses) *misses = ctl[msa::kCtlMisses];
+  if (copies) *copies = ctl[msa::kCtlMisses];
+  if (bytes) *bytes = ctl[msa::kCtlBytes];
   return MSA_OK;
 }
 
@@ -901,70 +916,23 @@ msa_status msa_fetch(msa_fetcher *f, const int32_t *ids, int32_t batch, int32_t 
                 f->max_batch, f->max_k);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaStream_t fst = reinterpret_cast<cudaStream_t>(fetch_stream);
-  const int n = batch * k;
-  MSA_CUDA(cudaMemcpyAsync(f->h_ids, ids, n * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
-  MSA_CUDA(cudaEventRecord(f->ev_ids, st));
-  MSA_CUDA(cudaEventSynchronize(f->ev_ids));
-  const int64_t now = ++f->stamp;
-  if (f->flags & MSA_FETCH_COLD) {
-    for (int s = 0; s < f->n_slots; ++s) {
-      if (f->slot_doc[s] >= 0) f->doc_slot[f->slot_doc[s]] = -1;
-      f->slot_doc[s] = -1;
-    }
-  }
   const msa_memory *mem = f->mem;
-  int n_miss = 0;
-  // resident documents keep their slots
-  for (int i = 0; i < n; ++i) {
-    const int d = f->h_ids[i];
-    if (d < 0 || d >= mem->n_docs) continue;
-    const int s = f->doc_slot[d];
-    if (s >= 0) f->slot_stamp[s] = now;
+  const int n = batch * k;
+  // slot assignment after the top-k (stream order), then the copies on the fetch stream
+  MSA_CUDA(launch_pdl(msa::fetch_assign_kernel, dim3(1), dim3(msa::kAssignThreads), 0, st, ids, n,
+                      mem->n_docs, static_cast<const int64_t *>(mem->d_doc_chunk_off),
+                      static_cast<int64_t>(f->row_bytes), static_cast<int64_t>(f->slot_bytes),
+                      f->n_slots, (f->flags & MSA_FETCH_COLD) ? 1 : 0, f->d_doc_slot, f->d_claim,
+                      f->d_slot_doc, f->d_slot_stamp, f->d_ctl, f->d_list, f->d_slots,
+                      f->d_scratch));
+  MSA_LAUNCHED("fetch_assign_kernel");
+  if (fst != st) {
+    MSA_CUDA(cudaEventRecord(f->ev_ids, st));
+    MSA_CUDA(cudaStreamWaitEvent(fst, f->ev_ids, 0));
   }
-  for (int i = 0; i < n; ++i) {
-    const int d = f->h_ids[i];
-    if (d < 0 || d >= mem->n_docs) {
-      f->h_slots[i] = 0;
-      continue;
-    }
-    int s = f->doc_slot[d];
-    if (s >= 0 && f->slot_stamp[s] == now) {
-      f->h_slots[i] = s;
-      ++f->hits;
-      continue;
-    }
-    // a clock over the slots this call has not claimed (n_slots >= n guarantees one)
-    while (f->slot_stamp[f->hand] == now) f->hand = (f->hand + 1) % f->n_slots;
-    s = f->hand;
-    f->hand = (f->hand + 1) % f->n_slots;
-    if (f->slot_doc[s] >= 0) f->doc_slot[f->slot_doc[s]] = -1;
-    f->slot_doc[s] = d;
-    f->doc_slot[d] = s;
-    f->slot_stamp[s] = now;
-    f->h_slots[i] = s;
-    const int64_t c0 = mem->doc_chunk_off[d], c1 = mem->doc_chunk_off[d + 1];
-    const size_t nb = static_cast<size_t>(c1 - c0) * f->row_bytes;
-    if (f->content_dev) {
-      f->h_list[3 * n_miss] = static_cast<int64_t>(c0) * static_cast<int64_t>(f->row_bytes);
-      f->h_list[3 * n_miss + 1] = static_cast<int64_t>(nb);
-      f->h_list[3 * n_miss + 2] = static_cast<int64_t>(s) * static_cast<int64_t>(f->slot_bytes);
-    } else {
-      MSA_CUDA(cudaMemcpyAsync(f->slot_cache + static_cast<size_t>(s) * f->slot_bytes,
-                               f->content_host + static_cast<size_t>(c0) * f->row_bytes, nb,
-                               cudaMemcpyHostToDevice, fst));
-    }
-    ++n_miss;
-    ++f->misses;
-    ++f->copies;
-    f->bytes += static_cast<int64_t>(nb);
-  }
-  MSA_CUDA(cudaMemcpyAsync(f->d_slots, f->h_slots, n * sizeof(int32_t), cudaMemcpyHostToDevice, fst));
-  if (f->content_dev && n_miss > 0) {
-    MSA_CUDA(cudaMemcpyAsync(f->d_list, f->h_list, static_cast<size_t>(n_miss) * 3 * 8,
-                             cudaMemcpyHostToDevice, fst));
-    msa::fetch_gather_kernel<<<n_miss, 256, 0, fst>>>(f->content_dev, f->slot_cache, f->d_list);
-    MSA_LAUNCHED("fetch_gather_kernel");
-  }
+  msa::fetch_gather_kernel<<<n, 256, 0, fst>>>(f->content_dev, f->slot_cache, f->d_list,
+                                                f->d_ctl);
+  MSA_LAUNCHED("fetch_gather_kernel");
   if (fst != st) {
     MSA_CUDA(cudaEventRecord(f->ev_fetch, fst));
     MSA_CUDA(cudaStreamWaitEvent(st, f->ev_fetch, 0));
@@ -1157,6 +1125,45 @@ msa_status msa_interleave_adaptive(const msa_memory *mem, const void *router_key
   if (stop_score != stop_score) return fail(MSA_ERR_INVALID_ARG, "stop_score is NaN");
   return interleave_impl(mem, router_keys, Qr, batch, tokens, k, max_rounds, stop_score, state,
                          taken, ids, scores, n_rounds, workspace, workspace_bytes, stream);
+}
+
+msa_status msa_topk_merge(const float *cand_scores, const int32_t *cand_ids, int32_t n_shards,
+                          int32_t batch, int32_t k_cand, const int32_t *shard_doc_base, int32_t k,
+                          int32_t *ids, float *scores, msa_stream stream) {
+  if (!cand_scores || !cand_ids || !shard_doc_base || !ids || !scores)
+    return fail(MSA_ERR_INVALID_ARG, "null argument");
+  if (n_shards < 1 || n_shards > msa::kMaxShards)
+    return fail(MSA_ERR_INVALID_ARG, "n_shards=%d must be in [1, %d]", n_shards, msa::kMaxShards);
+  if (k_cand < 1 || k_cand > msa::kMaxTopK)
+    return fail(MSA_ERR_INVALID_ARG, "k_cand=%d must be in [1, %d]", k_cand, msa::kMaxTopK);
+  if (static_cast<int64_t>(n_shards) * k_cand > msa::kTopkSlice)
+    return fail(MSA_ERR_UNSUPPORTED, "n_shards * k_cand = %d exceeds %d candidates",
+                n_shards * k_cand, msa::kTopkSlice);
+  if (k < 1 || k > msa::kMaxTopK || k > n_shards * k_cand)
+    return fail(MSA_ERR_INVALID_ARG, "k=%d must be in [1, min(%d, n_shards * k_cand)]", k,
+                msa::kMaxTopK);
+  if (batch < 1 || batch > 65535) return fail(MSA_ERR_INVALID_ARG, "batch=%d out of range", batch);
+  msa::ShardBases bases = {};
+  for (int s = 0; s < n_shards; ++s) {
+    if (shard_doc_base[s] < 0 || (s > 0 && shard_doc_base[s] < shard_doc_base[s - 1]))
+      return fail(MSA_ERR_INVALID_ARG, "shard_doc_base must be non-negative and non-decreasing");
+    bases.base[s] = shard_doc_base[s];
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define MSA_MERGE(KL)                                                                           \
+  MSA_CUDA(launch_pdl(msa::topk_merge_shards_kernel<KL>, dim3(batch), dim3(msa::kTopkThreads), \
+                      0, st, cand_scores, cand_ids, n_shards, batch, k_cand, bases, k, ids,     \
+                      scores));
+  if (k <= 16) {
+    MSA_MERGE(16)
+  } else if (k <= 32) {
+    MSA_MERGE(32)
+  } else {
+    MSA_MERGE(64)
+  }
+#undef MSA_MERGE
+  MSA_LAUNCHED("topk_merge_shards_kernel");
+  return MSA_OK;
 }
 
 msa_status msa_device_error(uint32_t *bits, msa_stream stream) {

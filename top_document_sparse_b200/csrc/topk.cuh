@@ -7,7 +7,8 @@
 // its slice's k largest keys (a memory of at most 2,048 documents: one
 // 128-thread CTA per query, no phase 2); phase 2 merges the slices'
 // candidates.  Both filter first (block_select_topk_fast) and sort only the
-// few survivors.
+// few survivors.  topk_merge_shards_kernel merges the candidates of several
+// memory shards (Memory Parallel).
 #pragma once
 #include "common.cuh"
 #include "ptx.cuh"
@@ -286,6 +287,52 @@ topk_merge_kernel(const unsigned long long *__restrict__ cand, int n_cand, int k
   for (int j = 0; j < kTopkPerThread; ++j) {
     const int i = warp * (32 * kTopkPerThread) + j * 32 + lane;
     key[j] = i < n_cand ? cand[static_cast<int64_t>(b) * n_cand + i] : 0ull;
+  }
+  block_select_topk_fast<KL>(key, k, wc, sel, wt, cbuf);
+  write_topk(sel, k, ids + static_cast<int64_t>(b) * k, scores + static_cast<int64_t>(b) * k);
+}
+
+// --- Memory Parallel ------------------------------------------------------------
+// The memory's documents are split into contiguous ranges (shards, one per GPU
+// in the pages' engine: Evermind summary sec. 4B "Memory Parallel & Tiered
+// Storage"; b-lab.team item 2); each shard routes its own documents and keeps
+// its top k_cand as (score, local id).  The global top-k is the k largest
+// (score, base + local id) keys over all shards' candidates: the global top-k
+// documents are each in their own shard's top k_cand (k_cand >= k), and the
+// keys order exactly as the single-memory top-k orders them, so the result is
+// bit-identical to routing the whole memory at once.
+constexpr int kMaxShards = 64;
+struct ShardBases {
+  int32_t base[kMaxShards];  // global id of each shard's document 0
+};
+
+// grid (B).  cand_* [n_shards][B][k_cand]; ids < 0 are padding.  n_shards *
+// k_cand <= kTopkSlice.
+template <int KL>
+__global__ void __launch_bounds__(kTopkThreads)
+topk_merge_shards_kernel(const float *__restrict__ cand_scores,
+                         const int32_t *__restrict__ cand_ids, int n_shards, int B, int k_cand,
+                         ShardBases bases, int k, int32_t *__restrict__ ids,
+                         float *__restrict__ scores) {
+  __shared__ unsigned long long wc[kTopkWarps * KL];
+  __shared__ unsigned long long sel[kMaxTopK];
+  __shared__ unsigned long long wt[kTopkWarps + 1], cbuf[kTopkCandCap];
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_wait();
+  griddep_launch();
+  const int n_cand = n_shards * k_cand;
+  unsigned long long key[kTopkPerThread];
+#pragma unroll
+  for (int j = 0; j < kTopkPerThread; ++j) {
+    const int i = warp * (32 * kTopkPerThread) + j * 32 + lane;
+    key[j] = 0ull;
+    if (i < n_cand) {
+      const int s = i / k_cand, r = i - s * k_cand;
+      const int64_t src = (static_cast<int64_t>(s) * B + b) * k_cand + r;
+      const int32_t id = cand_ids[src];
+      if (id >= 0) key[j] = topk_key(cand_scores[src], bases.base[s] + id);
+    }
   }
   block_select_topk_fast<KL>(key, k, wc, sel, wt, cbuf);
   write_topk(sel, k, ids + static_cast<int64_t>(b) * k, scores + static_cast<int64_t>(b) * k);

@@ -92,6 +92,8 @@ SIGNATURES = {
                                       _P]),
     "msa_interleave_adaptive": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, ctypes.c_float,
                                                _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "msa_topk_merge": (ctypes.c_int, [_P, _P, _I32, _I32, _I32, ctypes.POINTER(_I32), _I32, _P,
+                                      _P, _P]),
     "msa_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "msa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "msa_last_error": (ctypes.c_char_p, []),
@@ -352,6 +354,21 @@ class Fetcher:
                                   _ptr(V_tok), _ptr(O_tok), _stream(stream),
                                   _stream(fetch_stream) if fetch_stream is not None
                                   else _stream(stream)))
+
+
+def topk_merge(cand_scores, cand_ids, shard_doc_base, k: int, stream=None):
+    """Global top-k from every memory shard's candidates (msa_topk_merge).
+
+    cand_scores / cand_ids: device [n_shards][B][k_cand] (each shard's msa_route output, ids
+    local to the shard); shard_doc_base: the global id of each shard's document 0.  Returns
+    (ids [B][k] global, scores [B][k])."""
+    n_shards, B, kc = cand_ids.shape
+    base = (ctypes.c_int32 * n_shards)(*[int(x) for x in shard_doc_base])
+    ids = torch.empty(B, k, dtype=torch.int32, device=cand_ids.device)
+    scores = torch.empty(B, k, dtype=torch.float32, device=cand_ids.device)
+    _check(_lib.msa_topk_merge(_ptr(cand_scores), _ptr(cand_ids), n_shards, B, kc, base, k,
+                               _ptr(ids), _ptr(scores), _stream(stream)))
+    return ids, scores
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
