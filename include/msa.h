@@ -431,7 +431,61 @@ MSA_API msa_status msa_topk_merge(const float *cand_scores, const int32_t *cand_
                                   const int32_t *shard_doc_base, int32_t k, int32_t *ids,
                                   float *scores, msa_stream stream);
 
-/* Read and clear the device error word of the current device (synchronises/* Read and clear the device error word of the current device (synchronises
+/*
+ * Backward of the routing score [Evermind summary sec. 4A: continued
+ * pre-training supervises the router with an auxiliary routing loss L_aux; the
+ * training itself is outside this library].  For one routing call of `tokens`
+ * query rows with no carried state, doc_score[b][d] = max over tokens t and
+ * chunks c of document d of (1/H_r) sum_h cos(Qr[b,t,h], M[c,h]), M the pooled
+ * (un-normalised) router keys.  Given d_score = dL/d doc_score, the gradient
+ * of each document's max reaches its first maximising (token, chunk) pair, in
+ * (token, chunk) order:
+ *   d cos(q, m)/dq = m / (|q| |m|) - cos q / |q|^2   (and symmetrically for m;
+ *   a norm clamped at 1e-12 contributes no term).
+ *   router_mean   : device [C][H_r][d_r], msa_encode_memory's router_mean
+ *   Qr            : device [batch][tokens][H_r][d_r]
+ *   d_score       : device [batch][n_docs] fp32 (zeros skip their pairs)
+ *   d_Qr          : device [batch][tokens][H_r][d_r] fp32, overwritten
+ *   d_router_mean : device [C][H_r][d_r] fp32, overwritten
+ * The pooling's own backward (each chunk token receives d_router_mean / chunk
+ * length) is left to the caller.  CUDA-core kernel, one warp per (query,
+ * document) with a nonzero gradient.
+ */
+MSA_API msa_status msa_route_backward(const msa_memory *mem, const void *router_mean,
+                                      const void *Qr, int32_t batch, int32_t tokens,
+                                      const float *d_score, float *d_Qr, float *d_router_mean,
+                                      msa_stream stream);
+
+/*
+ * Backward of msa_sparse_attend [b-lab.team item 1 and stage "Sparse
+ * Generation"; the same context, masking, Global RoPE and GQA mapping].  With
+ * p = softmax(z) over the context rows of (b, i, h), z = <RoPE(Q), key> /
+ * sqrt(D), O = sum p value, and dO given:
+ *   dz = p (<dO, value> - <dO, O>);  dQ = RoPE^T(sum dz key) / sqrt(D);
+ *   dkey += dz RoPE(Q) / sqrt(D);    dvalue += p dO.
+ *   content, ids, Q, pos_offset, cache_capacity : as msa_sparse_attend
+ *   K_cache, V_cache : device [batch][cache_capacity][H_kv][D] as the forward
+ *                 left them (K rotated; the call's tokens appended)
+ *   cache_len0  : device [batch] int32, the lengths BEFORE the forward call
+ *   dO          : device [batch][tokens][n_q_heads][D]
+ *   dQ          : device fp32 [batch][tokens][n_q_heads][D], overwritten,
+ *                 with respect to Q before its RoPE
+ *   d_cache_k, d_cache_v : device fp32 [batch][cache_capacity][H_kv][D],
+ *                 overwritten, with respect to the cache rows as stored
+ *   d_content   : device fp32 [C][2][H_kv][D], overwritten, with respect to
+ *                 the pooled memory rows as stored
+ * n_q_heads <= 32.  CUDA-core kernel, one warp per (query, token, head).
+ */
+MSA_API msa_status msa_sparse_attend_backward(const msa_memory *mem, const void *content,
+                                              const int32_t *ids, int32_t batch, int32_t k,
+                                              int32_t tokens, int32_t n_q_heads, const void *Q,
+                                              const void *K_cache, const void *V_cache,
+                                              const int32_t *cache_len0, int32_t cache_capacity,
+                                              int32_t pos_offset, const void *dO, float *dQ,
+                                              float *d_cache_k, float *d_cache_v,
+                                              float *d_content, msa_stream stream);
+
+/* Read and clear the device error word of the current device (synchronises/* Read and clear the device error word of the current device (synchronises/* Read and clear the device error word of the current device (synchronises
  * `stream`).  *bits receives the MSA_DEVERR_* bits; returns MSA_ERR_TIMEOUT or
  * MSA_ERR_STATE when a bit was set, else MSA_OK. */
 MSA_API msa_status msa_device_error(uint32_t *bits, msa_stream stream);

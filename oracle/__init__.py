@@ -80,6 +80,17 @@ def _load():
                                           _i64p, _i32p, ctypes.c_int32, ctypes.c_int32,
                                           ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
                                           _dp, _dp, _dp]
+        lib.msa_oracle_route_backward.restype = None
+        lib.msa_oracle_route_backward.argtypes = [_dp, ctypes.c_int32, ctypes.c_int32, _dp, _i64p,
+                                                  ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                  _dp, _dp, _dp]
+        lib.msa_oracle_attend_backward.restype = None
+        lib.msa_oracle_attend_backward.argtypes = [_dp, ctypes.c_int32, ctypes.c_int32,
+                                                   ctypes.c_int32, _dp, _dp, ctypes.c_int32,
+                                                   ctypes.c_int32, _dp, _dp, _i64p, _i32p,
+                                                   ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                   ctypes.c_int32, ctypes.c_double, _dp,
+                                                   ctypes.c_int64, _dp, _dp, _dp, _dp, _dp]
         _lib = lib
     return _lib
 
@@ -271,3 +282,49 @@ def interleave(Qr, Krbar, doc_chunk_off, k: int, rounds: int, stop_score=None):
     if stop_score is not None:
         return out, state, n_rounds
     return out
+
+
+def route_backward(Qr, Krbar, doc_chunk_off, G):
+    """Gradients of sum_{b,d} G[b,d] * doc_score[b,d] (one routing call, no carried state) with
+    respect to the query router rows and the pooled router keys: (dQr [B][T][H_r][d_r],
+    dKrbar [C][H_r][d_r]).  The gradient of a max reaches its maximising (token, chunk) pair,
+    the first in (token, chunk) order among equal maxima."""
+    Q = f64(Qr)
+    if Q.ndim == 3:
+        Q = Q[:, None]
+    B, T, H_r, d_r = Q.shape
+    K = f64(Krbar)
+    off = _i64(doc_chunk_off)
+    g = f64(G)
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    _load().msa_oracle_route_backward(_p(Q, _dp), B, T, _p(K, _dp), _p(off, _i64p), off.size - 1,
+                                      H_r, d_r, _p(g, _dp), _p(dQ, _dp), _p(dK, _dp))
+    return dQ, dK
+
+
+def attend_backward(Q, K_loc, V_loc, q_start: int, Kbar, Vbar, doc_chunk_off, ids,
+                    pos_offset: int, theta: float, dO):
+    """Gradients of sum(dO * O) for the attention of ``attend`` with respect to Q (before RoPE),
+    the local keys (before RoPE) and values, and the pooled memory rows Kbar / Vbar:
+    (dQ, dK_loc, dV_loc, dKbar, dVbar)."""
+    Q, Kl, Vl, g = f64(Q), f64(K_loc), f64(V_loc), f64(dO)
+    B, T, H_q, D = Q.shape
+    _, L_loc, H_kv, _ = Kl.shape
+    if q_start + T > L_loc:
+        raise ValueError("local history shorter than q_start + T")
+    Kb, Vb = f64(Kbar), f64(Vbar)
+    off = _i64(doc_chunk_off)
+    idx = _i32(ids)
+    k = idx.shape[1]
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(Kl)
+    dV = np.zeros_like(Vl)
+    dKb = np.zeros_like(Kb)
+    dVb = np.zeros_like(Vb)
+    _load().msa_oracle_attend_backward(_p(Q, _dp), B, T, H_q, _p(Kl, _dp), _p(Vl, _dp), L_loc,
+                                       q_start, _p(Kb, _dp), _p(Vb, _dp), _p(off, _i64p),
+                                       _p(idx, _i32p), k, H_kv, D, pos_offset, theta, _p(g, _dp),
+                                       Kb.shape[0], _p(dQ, _dp), _p(dK, _dp), _p(dV, _dp),
+                                       _p(dKb, _dp), _p(dVb, _dp))
+    return dQ, dK, dV, dKb, dVb

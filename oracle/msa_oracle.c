@@ -320,3 +320,205 @@ void msa_oracle_attend(const double *Q, int32_t B, int32_t T, int32_t H_q,
       free(key);
     }
 }
+
+/* ---------------------------------------------------------------------------
+ * Backward of the routing score, for training the router with an auxiliary
+ * routing loss [EVM sec. 4A: the router is supervised with L_aux during
+ * continued pre-training].  For one routing call (no carried state):
+ *   doc_score[b][d] = max over tokens t and chunks c of d of
+ *                     s(b,t,c) = (1/H_r) sum_h cos(Qr[b,t,h], Krbar[c,h]),
+ * so, given dL/d doc_score = G[b][d], the gradient flows to the maximising
+ * pair (t*, c*) only -- the first in (t ascending, c ascending) order among
+ * equal maxima -- and there:
+ *   d cos(q, k) / dq = k / (|q| |k|) - cos(q, k) q / |q|^2   (|q|, |k| > eps;
+ *   a norm clamped at eps is a constant: its term drops),
+ * and symmetrically for k.  dQr and dKrbar are overwritten.
+ * ------------------------------------------------------------------------- */
+static void cosine_grad(const double *q, const double *k, int32_t n, double g,
+                        double *dq, double *dk) {
+  double dot = 0.0, qq = 0.0, kk = 0.0;
+  for (int32_t i = 0; i < n; ++i) {
+    dot += q[i] * k[i];
+    qq += q[i] * q[i];
+    kk += k[i] * k[i];
+  }
+  const double rq = sqrt(qq), rk = sqrt(kk);
+  const double nq = rq < ORACLE_EPS ? ORACLE_EPS : rq;
+  const double nk = rk < ORACLE_EPS ? ORACLE_EPS : rk;
+  const double c = dot / (nq * nk);
+  for (int32_t i = 0; i < n; ++i) {
+    double gq = k[i] / (nq * nk), gk = q[i] / (nq * nk);
+    if (rq >= ORACLE_EPS) gq -= c * q[i] / (nq * nq);
+    if (rk >= ORACLE_EPS) gk -= c * k[i] / (nk * nk);
+    dq[i] += g * gq;
+    dk[i] += g * gk;
+  }
+}
+
+void msa_oracle_route_backward(const double *Qr, int32_t B, int32_t T,
+                               const double *Krbar, const int64_t *doc_chunk_off,
+                               int32_t n_docs, int32_t H_r, int32_t d_r,
+                               const double *G, double *dQr, double *dKrbar) {
+  const int64_t wr = (int64_t)H_r * d_r;
+  memset(dQr, 0, sizeof(double) * (size_t)B * T * wr);
+  memset(dKrbar, 0, sizeof(double) * (size_t)doc_chunk_off[n_docs] * wr);
+  for (int32_t b = 0; b < B; ++b)
+    for (int32_t d = 0; d < n_docs; ++d) {
+      const double g = G[(int64_t)b * n_docs + d];
+      if (g == 0.0 || T < 1 || doc_chunk_off[d + 1] == doc_chunk_off[d]) continue;
+      double best = -INFINITY;
+      int32_t tb = 0;
+      int64_t cb = doc_chunk_off[d];
+      for (int32_t t = 0; t < T; ++t)
+        for (int64_t c = doc_chunk_off[d]; c < doc_chunk_off[d + 1]; ++c) {
+          const double s = msa_oracle_chunk_score(Qr + ((int64_t)b * T + t) * wr,
+                                                  Krbar + c * wr, H_r, d_r);
+          if (s > best) {
+            best = s;
+            tb = t;
+            cb = c;
+          }
+        }
+      for (int32_t h = 0; h < H_r; ++h)
+        cosine_grad(Qr + ((int64_t)b * T + tb) * wr + (int64_t)h * d_r,
+                    Krbar + cb * wr + (int64_t)h * d_r, d_r, g / (double)H_r,
+                    dQr + ((int64_t)b * T + tb) * wr + (int64_t)h * d_r,
+                    dKrbar + cb * wr + (int64_t)h * d_r);
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Backward of the sparse attention [BLAB stage "Sparse Generation"; the same
+ * context and masking as msa_oracle_attend].  With p = softmax(z) over the
+ * context rows y of (b, i, h), z_y = scale * <q', key_y>, q' = RoPE(Q) and
+ * O = sum_y p_y value_y, given dO:
+ *   dp_y  = <dO, value_y>,        Dv = <dO, O> = sum_y p_y dp_y
+ *   dz_y  = p_y (dp_y - Dv)
+ *   dq'  += scale dz_y key_y;     dQ = RoPE^-1(dq') (the rotation's transpose)
+ *   dkey_y += scale dz_y q';      dvalue_y += p_y dO
+ * Memory rows accumulate into dKbar / dVbar [C][H_kv][D] (keys as stored:
+ * pooled after document-wise RoPE); local rows into dK_loc / dV_loc
+ * [B][L_loc][H_kv][D], dK_loc with respect to the keys BEFORE their RoPE at
+ * pos_offset + l (the inputs of msa_oracle_attend).  Every output is
+ * overwritten (dKbar / dVbar: n_chunks rows).  Plain loops, no parallelism
+ * (outputs are shared).
+ * ------------------------------------------------------------------------- */
+static void rope_vec_inverse(double *x, int32_t dim, double p, double theta) {
+  rope_vec(x, dim, -p, theta);  /* a rotation by -angle is the transpose */
+}
+
+void msa_oracle_attend_backward(const double *Q, int32_t B, int32_t T, int32_t H_q,
+                                const double *K_loc, const double *V_loc, int32_t L_loc,
+                                int32_t q_start, const double *Kbar, const double *Vbar,
+                                const int64_t *doc_chunk_off, const int32_t *ids,
+                                int32_t k, int32_t H_kv, int32_t D, int32_t pos_offset,
+                                double theta, const double *dO, int64_t n_chunks, double *dQ,
+                                double *dK_loc, double *dV_loc, double *dKbar, double *dVbar) {
+  const int32_t group = H_q / H_kv;
+  const double scale = 1.0 / sqrt((double)D);
+  memset(dQ, 0, sizeof(double) * (size_t)B * T * H_q * D);
+  memset(dK_loc, 0, sizeof(double) * (size_t)B * L_loc * H_kv * D);
+  memset(dV_loc, 0, sizeof(double) * (size_t)B * L_loc * H_kv * D);
+  memset(dKbar, 0, sizeof(double) * (size_t)n_chunks * H_kv * D);
+  memset(dVbar, 0, sizeof(double) * (size_t)n_chunks * H_kv * D);
+  for (int32_t b = 0; b < B; ++b)
+    for (int32_t i = 0; i < T; ++i) {
+      const int32_t j = q_start + i;
+      int64_t n_mem = 0;
+      for (int32_t r = 0; r < k; ++r) {
+        const int32_t d = ids[(int64_t)b * k + r];
+        n_mem += doc_chunk_off[d + 1] - doc_chunk_off[d];
+      }
+      const int64_t n_ctx = n_mem + (int64_t)j + 1;
+      double *z = (double *)malloc(sizeof(double) * n_ctx);
+      double **key = (double **)malloc(sizeof(double *) * n_ctx);
+      double **val = (double **)malloc(sizeof(double *) * n_ctx);
+      double **dkey = (double **)malloc(sizeof(double *) * n_ctx);
+      double **dval = (double **)malloc(sizeof(double *) * n_ctx);
+      double *rot = (double *)malloc(sizeof(double) * ((size_t)j + 1) * D);
+      double *drot = (double *)malloc(sizeof(double) * ((size_t)j + 1) * D);
+      double *q = (double *)malloc(sizeof(double) * D);
+      double *dq = (double *)malloc(sizeof(double) * D);
+      double *o = (double *)malloc(sizeof(double) * D);
+      for (int32_t h = 0; h < H_q; ++h) {
+        const int32_t g = h / group;
+        /* the context rows, in the forward's order */
+        int64_t x = 0;
+        for (int32_t r = 0; r < k; ++r) {
+          const int32_t d = ids[(int64_t)b * k + r];
+          for (int64_t c = doc_chunk_off[d]; c < doc_chunk_off[d + 1]; ++c) {
+            key[x] = (double *)(Kbar + (c * H_kv + g) * (int64_t)D);
+            val[x] = (double *)(Vbar + (c * H_kv + g) * (int64_t)D);
+            dkey[x] = dKbar + (c * H_kv + g) * (int64_t)D;
+            dval[x] = dVbar + (c * H_kv + g) * (int64_t)D;
+            ++x;
+          }
+        }
+        for (int32_t l = 0; l <= j; ++l) {
+          double *kr = rot + (int64_t)l * D;
+          memcpy(kr, K_loc + (((int64_t)b * L_loc + l) * H_kv + g) * D, sizeof(double) * D);
+          rope_vec(kr, D, (double)(pos_offset + l), theta);
+          memset(drot + (int64_t)l * D, 0, sizeof(double) * D);
+          key[x] = kr;
+          val[x] = (double *)(V_loc + (((int64_t)b * L_loc + l) * H_kv + g) * D);
+          dkey[x] = drot + (int64_t)l * D;
+          dval[x] = dV_loc + (((int64_t)b * L_loc + l) * H_kv + g) * D;
+          ++x;
+        }
+        memcpy(q, Q + (((int64_t)b * T + i) * H_q + h) * D, sizeof(double) * D);
+        rope_vec(q, D, (double)(pos_offset + j), theta);
+        /* forward: p and O */
+        double m = -INFINITY;
+        for (int64_t y = 0; y < n_ctx; ++y) {
+          double dot = 0.0;
+          for (int32_t e = 0; e < D; ++e) dot += q[e] * key[y][e];
+          z[y] = dot * scale;
+          if (z[y] > m) m = z[y];
+        }
+        double sum = 0.0;
+        for (int64_t y = 0; y < n_ctx; ++y) {
+          z[y] = exp(z[y] - m);
+          sum += z[y];
+        }
+        for (int32_t e = 0; e < D; ++e) o[e] = 0.0;
+        for (int64_t y = 0; y < n_ctx; ++y) {
+          z[y] /= sum;
+          for (int32_t e = 0; e < D; ++e) o[e] += z[y] * val[y][e];
+        }
+        /* backward */
+        const double *go = dO + (((int64_t)b * T + i) * H_q + h) * D;
+        double Dv = 0.0;
+        for (int32_t e = 0; e < D; ++e) Dv += go[e] * o[e];
+        for (int32_t e = 0; e < D; ++e) dq[e] = 0.0;
+        for (int64_t y = 0; y < n_ctx; ++y) {
+          double dp = 0.0;
+          for (int32_t e = 0; e < D; ++e) dp += go[e] * val[y][e];
+          const double dz = z[y] * (dp - Dv);
+          for (int32_t e = 0; e < D; ++e) {
+            dq[e] += scale * dz * key[y][e];
+            dkey[y][e] += scale * dz * q[e];
+            dval[y][e] += z[y] * go[e];
+          }
+        }
+        rope_vec_inverse(dq, D, (double)(pos_offset + j), theta);
+        memcpy(dQ + (((int64_t)b * T + i) * H_q + h) * D, dq, sizeof(double) * D);
+        /* local keys: back through their RoPE */
+        for (int32_t l = 0; l <= j; ++l) {
+          double *dr = drot + (int64_t)l * D;
+          rope_vec_inverse(dr, D, (double)(pos_offset + l), theta);
+          double *dst = dK_loc + (((int64_t)b * L_loc + l) * H_kv + g) * D;
+          for (int32_t e = 0; e < D; ++e) dst[e] += dr[e];
+        }
+      }
+      free(z);
+      free(key);
+      free(val);
+      free(dkey);
+      free(dval);
+      free(rot);
+      free(drot);
+      free(q);
+      free(dq);
+      free(o);
+    }
+}

@@ -12,6 +12,7 @@
 #include <utility>
 
 #include "attend.cuh"
+#include "backward.cuh"
 #include "common.cuh"
 #include "pool.cuh"
 #include "route.cuh"
@@ -918,6 +919,17 @@ msa_status msa_fetch(msa_fetcher *f, const int32_t *ids, int32_t batch, int32_t 
   cudaStream_t fst = reinterpret_cast<cudaStream_t>(fetch_stream);
   const msa_memory *mem = f->mem;
   const int n = batch * k;
+  // The fetch kernels prefer the largest shared-memory carveout (they use no shared memory):
+  // an SM runs CTAs of one L1 / shared-memory split at a time, and the route kernel's split
+  // is the largest, so with the same preference a fetch can run on the SMs beside it.
+  static std::once_flag carveout;
+  std::call_once(carveout, [] {
+    cudaFuncSetAttribute(msa::fetch_assign_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+    cudaFuncSetAttribute(msa::fetch_gather_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+    cudaGetLastError();
+  });
   // slot assignment after the top-k (stream order), then the copies on the fetch stream
   MSA_CUDA(launch_pdl(msa::fetch_assign_kernel, dim3(1), dim3(msa::kAssignThreads), 0, st, ids, n,
                       mem->n_docs, static_cast<const int64_t *>(mem->d_doc_chunk_off),
@@ -1163,6 +1175,72 @@ msa_status msa_topk_merge(const float *cand_scores, const int32_t *cand_ids, int
   }
 #undef MSA_MERGE
   MSA_LAUNCHED("topk_merge_shards_kernel");
+  return MSA_OK;
+}
+
+msa_status msa_route_backward(const msa_memory *mem, const void *router_mean, const void *Qr,
+                              int32_t batch, int32_t tokens, const float *d_score, float *d_Qr,
+                              float *d_router_mean, msa_stream stream) {
+  if (!mem || !router_mean || !Qr || !d_score || !d_Qr || !d_router_mean)
+    return fail(MSA_ERR_INVALID_ARG, "null argument");
+  if (batch < 1 || tokens < 1) return fail(MSA_ERR_INVALID_ARG, "batch and tokens must be >= 1");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t W = static_cast<int64_t>(mem->H_r) * mem->d_r;
+  MSA_CUDA(cudaMemsetAsync(d_Qr, 0, static_cast<size_t>(batch) * tokens * W * 4, st));
+  MSA_CUDA(cudaMemsetAsync(d_router_mean, 0, static_cast<size_t>(mem->n_chunks) * W * 4, st));
+  const int64_t warps = static_cast<int64_t>(batch) * mem->n_docs;
+  const unsigned grid =
+      static_cast<unsigned>(std::min<int64_t>((warps + 7) / 8, static_cast<int64_t>(num_sms()) * 8));
+  if (mem->dtype == MSA_BF16)
+    msa::route_backward_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(Qr), batch, tokens,
+        static_cast<const __nv_bfloat16 *>(router_mean), mem->d_doc_chunk_off, mem->n_docs,
+        mem->H_r, mem->d_r, d_score, d_Qr, d_router_mean);
+  else
+    msa::route_backward_kernel<float><<<grid, 256, 0, st>>>(
+        static_cast<const float *>(Qr), batch, tokens, static_cast<const float *>(router_mean),
+        mem->d_doc_chunk_off, mem->n_docs, mem->H_r, mem->d_r, d_score, d_Qr, d_router_mean);
+  MSA_LAUNCHED("route_backward_kernel");
+  return MSA_OK;
+}
+
+msa_status msa_sparse_attend_backward(const msa_memory *mem, const void *content,
+                                      const int32_t *ids, int32_t batch, int32_t k,
+                                      int32_t tokens, int32_t n_q_heads, const void *Q,
+                                      const void *K_cache, const void *V_cache,
+                                      const int32_t *cache_len0, int32_t cache_capacity,
+                                      int32_t pos_offset, const void *dO, float *dQ,
+                                      float *d_cache_k, float *d_cache_v, float *d_content,
+                                      msa_stream stream) {
+  const msa_status chk =
+      attend_shape_check(mem, batch, k, tokens, n_q_heads, cache_capacity, pos_offset);
+  if (chk != MSA_OK) return chk;
+  if (n_q_heads > 32)
+    return fail(MSA_ERR_UNSUPPORTED, "the attention backward takes at most 32 query heads");
+  if (!content || (k > 0 && !ids) || !Q || !K_cache || !V_cache || !cache_len0 || !dO || !dQ ||
+      !d_cache_k || !d_cache_v || !d_content)
+    return fail(MSA_ERR_INVALID_ARG, "null pointer argument");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t row = static_cast<size_t>(mem->H_kv) * mem->D * 4;
+  MSA_CUDA(cudaMemsetAsync(d_content, 0, static_cast<size_t>(mem->n_chunks) * 2 * row, st));
+  MSA_CUDA(cudaMemsetAsync(d_cache_k, 0, static_cast<size_t>(batch) * cache_capacity * row, st));
+  MSA_CUDA(cudaMemsetAsync(d_cache_v, 0, static_cast<size_t>(batch) * cache_capacity * row, st));
+  const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(mem->D)));
+  const dim3 grid(static_cast<unsigned>(static_cast<int64_t>(batch) * tokens));
+  const dim3 block(static_cast<unsigned>(n_q_heads * 32));
+#define MSA_ATT_BWD(T, DD)                                                                          \
+  msa::attend_backward_kernel<T, DD><<<grid, block, 0, st>>>(                                      \
+      static_cast<const T *>(content), ids, k, mem->d_doc_chunk_off, mem->n_docs, mem->H_kv,      \
+      n_q_heads, static_cast<const T *>(Q), tokens, static_cast<const T *>(K_cache),              \
+      static_cast<const T *>(V_cache), cache_len0, cache_capacity, pos_offset, mem->d_rope, scale, \
+      static_cast<const T *>(dO), dQ, d_content, d_cache_k, d_cache_v);
+  if (mem->dtype == MSA_BF16) {
+    if (mem->D == 128) { MSA_ATT_BWD(__nv_bfloat16, 128) } else { MSA_ATT_BWD(__nv_bfloat16, 64) }
+  } else {
+    if (mem->D == 128) { MSA_ATT_BWD(float, 128) } else { MSA_ATT_BWD(float, 64) }
+  }
+#undef MSA_ATT_BWD
+  MSA_LAUNCHED("attend_backward_kernel");
   return MSA_OK;
 }
 

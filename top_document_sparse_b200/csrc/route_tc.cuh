@@ -127,7 +127,12 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     }
   }
   griddep_wait();  // setup above overlaps the previous kernel's drain
-  griddep_launch();
+  // The next kernel (the top-k) may be scheduled once every CTA has started the
+  // epilogue of its last tile (see the epilogue loop), not earlier: its CTAs
+  // only wait for this kernel, and resident early they would hold every SM's
+  // spare threads and registers for the whole stream, so that no other work
+  // (a fetch on another stream) could run beside it.  With one tile per CTA
+  // (the 1M-token decode) that is at once.
 
   auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
     if (*fail) return false;
@@ -222,6 +227,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     const int tid = threadIdx.x;  // 0..127 == TMEM lane == chunk row of the tile
     int tl = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tl) {
+      if (tile + static_cast<int>(gridDim.x) >= n_tiles) griddep_launch();  // the last tile
       const int rt = tile / n_chunk_tiles, ct = tile % n_chunk_tiles;
       const int buf = tl & 1;
       const int64_t c0 = static_cast<int64_t>(ct) * L::kTileC;

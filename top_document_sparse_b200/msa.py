@@ -94,6 +94,9 @@ SIGNATURES = {
                                                _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "msa_topk_merge": (ctypes.c_int, [_P, _P, _I32, _I32, _I32, ctypes.POINTER(_I32), _I32, _P,
                                       _P, _P]),
+    "msa_route_backward": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _P, _P, _P, _P]),
+    "msa_sparse_attend_backward": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _P, _P,
+                                                  _P, _P, _I32, _I32, _P, _P, _P, _P, _P, _P]),
     "msa_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "msa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "msa_last_error": (ctypes.c_char_p, []),
@@ -283,6 +286,33 @@ class Memory:
                                             _ptr(taken), _ptr(ids), _ptr(scores), _ptr(n_rounds),
                                             _ptr(ws), ws.numel(), _stream(stream)))
         return ids, scores, state, taken, n_rounds
+
+    def route_backward(self, router_mean, Qr, d_score, stream=None):
+        """Gradients of sum(d_score * doc_score) of one routing call of Qr [B][T][H_r][d_r]
+        (msa_route_backward): (d_Qr, d_router_mean), fp32."""
+        B, T = Qr.shape[0], Qr.shape[1]
+        dQr = torch.empty(Qr.shape, dtype=torch.float32, device=Qr.device)
+        dM = torch.empty(router_mean.shape, dtype=torch.float32, device=Qr.device)
+        _check(_lib.msa_route_backward(self.handle, _ptr(router_mean), _ptr(Qr), B, T,
+                                       _ptr(d_score), _ptr(dQr), _ptr(dM), _stream(stream)))
+        return dQr, dM
+
+    def sparse_attend_backward(self, content, ids, Q, K_cache, V_cache, cache_len0,
+                               pos_offset: int, dO, stream=None):
+        """Gradients of sum(dO * O) of a msa_sparse_attend call (msa_sparse_attend_backward):
+        (dQ, d_cache_k, d_cache_v, d_content), fp32."""
+        B, T, H_q, _ = Q.shape
+        k = ids.shape[1] if ids is not None else 0
+        dev = Q.device
+        dQ = torch.empty(Q.shape, dtype=torch.float32, device=dev)
+        dKc = torch.empty(K_cache.shape, dtype=torch.float32, device=dev)
+        dVc = torch.empty(V_cache.shape, dtype=torch.float32, device=dev)
+        dC = torch.empty(content.shape, dtype=torch.float32, device=dev)
+        _check(_lib.msa_sparse_attend_backward(
+            self.handle, _ptr(content), _ptr(ids), B, k, T, H_q, _ptr(Q), _ptr(K_cache),
+            _ptr(V_cache), _ptr(cache_len0), K_cache.shape[1], pos_offset, _ptr(dO), _ptr(dQ),
+            _ptr(dKc), _ptr(dVc), _ptr(dC), _stream(stream)))
+        return dQ, dKc, dVc, dC
 
     def step_workspace_size(self, batch: int, k: int, n_q_heads: int) -> int:
         return _lib.msa_step_workspace_size(self.handle, batch, k, n_q_heads)
