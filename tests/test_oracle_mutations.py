@@ -18,7 +18,10 @@ import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "msa_oracle.c")
 
-# (name, [(original text, mutated text), ...]); each original text occurs exactly once
+# (name, [(original text, mutated text), ...]); each original text occurs exactly once in the
+# forward part of the source (everything before the gradients, which the pins here do not call;
+# tests/test_oracle_backward.py pins those by finite differences)
+BACKWARD_START = "\nvoid msa_oracle_route_backward("
 MUTANTS = [
     ("rope_rotation_sign", [("    x[i] = a * c - b * s;", "    x[i] = a * c + b * s;")]),
     ("rope_adjacent_pairs", [("    double a = x[i], b = x[i + half];",
@@ -72,9 +75,12 @@ def workdir():
 
 def _build_mutant(workdir, name, edits):
     src = open(SRC).read()
+    cut = src.index(BACKWARD_START)
+    fwd, bwd = src[:cut], src[cut:]
     for old, new in edits:
-        assert src.count(old) == 1, f"{name}: pattern must occur once: {old!r}"
-        src = src.replace(old, new)
+        assert fwd.count(old) == 1, f"{name}: pattern must occur once: {old!r}"
+        fwd = fwd.replace(old, new)
+    src = fwd + bwd
     c_path = os.path.join(workdir, f"{name}.c")
     so_path = os.path.join(workdir, f"{name}.so")
     with open(c_path, "w") as f:
