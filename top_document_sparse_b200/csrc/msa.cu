@@ -363,35 +363,36 @@ msa_status launch_attend_mma(const msa_memory *mem, const void *content, const i
                              const AttendPlan &plan, void *O, void *ws, cudaStream_t st) {
   const float scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)) * 1.4426950408889634);
   if constexpr (D == 128) {
-   if (T > 1) {
-    // several tokens (prefill), tensor cores: one CTA per (query, kv head, tile of 128 / G
-    // tokens x G heads); append_kernel ran before
     using Pt = msa::PtcSmem<D>;
     const int smem_pt = Pt::bytes(plan.table_cap);
-    if (smem_pt > max_dyn_smem())
-      return fail(MSA_ERR_UNSUPPORTED, "prefill needs %d B of shared memory", smem_pt);
-    auto kpt = msa::attend_prefill_tc_kernel<128, G>;
-    MSA_CUDA(cudaFuncSetAttribute(kpt, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_pt));
-    constexpr int TT = msa::kPtcRows / G;
-    dim3 grid_pt(static_cast<unsigned>(B * mem->H_kv), static_cast<unsigned>((T + TT - 1) / TT));
-    if (grid_pt.y > 65535) return fail(MSA_ERR_UNSUPPORTED, "too many query tokens");
-    MSA_CUDA(launch_pdl(kpt, grid_pt, dim3(msa::kPtcThreads), smem_pt, st,
-                        static_cast<const __nv_bfloat16 *>(content), ids, k,
-                        static_cast<const int64_t *>(mem->d_doc_chunk_off), mem->n_docs, slots,
-                        slot_chunks, mem->H_kv, static_cast<const __nv_bfloat16 *>(Q), T,
-                        static_cast<const __nv_bfloat16 *>(Kc), static_cast<const __nv_bfloat16 *>(Vc),
-                        static_cast<const int32_t *>(cache_len), cap, pos_offset,
-                        static_cast<const float2 *>(mem->d_rope), scale_log2, plan.table_cap,
-                        static_cast<__nv_bfloat16 *>(O)));
-    MSA_LAUNCHED("attend_prefill_tc_kernel");
-    MSA_CUDA(launch_pdl(msa::advance_kernel, dim3((B + 255) / 256), dim3(256), 0, st, cache_len, B,
-                        T, cap));
-    MSA_LAUNCHED("advance_kernel");
-    return MSA_OK;
-   }
+    if (T > 1 && smem_pt <= max_dyn_smem()) {
+      // several tokens (prefill), tensor cores: one CTA per (query, kv head, pair of adjacent
+      // tiles of 128 / G tokens x G heads); append_kernel ran before
+      auto kpt = msa::attend_prefill_tc_kernel<128, G>;
+      MSA_CUDA(cudaFuncSetAttribute(kpt, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_pt));
+      constexpr int TT = msa::kPtcRows / G;
+      const int n_tiles = (T + TT - 1) / TT;
+      dim3 grid_pt(static_cast<unsigned>(B * mem->H_kv), static_cast<unsigned>((n_tiles + 1) / 2));
+      if (grid_pt.y > 65535) return fail(MSA_ERR_UNSUPPORTED, "too many query tokens");
+      MSA_CUDA(launch_pdl(kpt, grid_pt, dim3(msa::kPtcThreads), smem_pt, st,
+                          static_cast<const __nv_bfloat16 *>(content), ids, k,
+                          static_cast<const int64_t *>(mem->d_doc_chunk_off), mem->n_docs, slots,
+                          slot_chunks, mem->H_kv, static_cast<const __nv_bfloat16 *>(Q), T,
+                          static_cast<const __nv_bfloat16 *>(Kc),
+                          static_cast<const __nv_bfloat16 *>(Vc),
+                          static_cast<const int32_t *>(cache_len), cap, pos_offset,
+                          static_cast<const float2 *>(mem->d_rope), scale_log2, plan.table_cap,
+                          static_cast<__nv_bfloat16 *>(O)));
+      MSA_LAUNCHED("attend_prefill_tc_kernel");
+      MSA_CUDA(launch_pdl(msa::advance_kernel, dim3((B + 255) / 256), dim3(256), 0, st, cache_len,
+                          B, T, cap));
+      MSA_LAUNCHED("advance_kernel");
+      return MSA_OK;
+    }
   }
   if (T > 1) {
-    // several tokens (prefill), head_dim 64: one CTA per (query, kv head, tile of 4 x 16 / G
+    // several tokens (prefill) on mma.sync (head_dim 64, or a chunk table too large for the
+    // tensor-core kernel's shared memory): one CTA per (query, kv head, tile of 4 x 16 / G
     // tokens) shares each staged context block between its tokens; append_kernel ran before
     using Pf = msa::PfSmem<D>;
     const int smem_pf = Pf::bytes(plan.table_cap);

@@ -1,32 +1,46 @@
 // prefill_tc.cuh -- multi-token (prefill) sparse GQA attention on the
 // 5th-generation tensor cores (MSA, b-lab.team summary item 1 "Scalable Sparse
 // Attention" and "Global RoPE", stage "Sparse Generation"): the call's tokens
-// attend over [pooled K/V of the retrieved documents' chunks, rank order, all
-// visible] ++ [local cache rows, causal: token t sees local rows up to
-// cache_len + t], with Q rotated at pos_offset + cache_len + t.
+// attend over [pooled K/V of the retrieved documents' chunks, all visible] ++
+// [local cache rows, causal: token t sees local rows up to cache_len + t],
+// with Q rotated at pos_offset + cache_len + t.
 //
-// One CTA per (query, kv head, tile of 128 query rows); a row is a (token,
-// query head of the GQA group) pair, so a tile holds 128 / G tokens.  The
-// context streams through in blocks of 64 rows:
+// One CTA per (query, kv head, pair of adjacent tiles of 128 query rows); a
+// row is a (token, query head of the GQA group) pair, so a tile holds 128 / G
+// tokens.  Both tiles share every K/V block the CTA loads.  The context
+// streams through in blocks of 64 rows, the local cache blocks first (their
+// rows need no chunk table, so the first loads start at once), then the
+// retrieved chunks; the online softmax does not depend on the order.  Per tile
+// and block:
 //   S   = Q K^T           tcgen05.mma, M = 128 query rows, N = 64 context
 //                          rows, K = D; Q and the K block in shared memory
-//                          (K-major, 128-byte swizzle), S in TMEM
-//   P   = exp2(S - m)     the four softmax warps: warp w reads TMEM lanes
-//                          32w..32w+31 (thread = query row), masks, keeps the
-//                          row's reference max m and sum l, writes P as bf16
-//                          to shared memory (K-major; over the block's K
-//                          rows, dead once S is computed) and, when the row's
-//                          max rises more than 8 (log2 units) above m, moves
-//                          m and rescales its row of O in TMEM; below that P
-//                          stays under 2^8 and the result is the same
+//                          (K-major, 128-byte swizzle); S in one of two TMEM
+//                          buffers, so Q K^T of a later block runs while the
+//                          softmax works on this one
+//   P   = exp2(S - m)     the tile's four softmax warps: warp w reads TMEM
+//                          lanes 32 (w % 4) .. (thread = query row), masks the
+//                          diagonal and ragged blocks, keeps the row's
+//                          reference max m and sum l, writes P as bf16 to the
+//                          tile's P buffer and, when the row's max rises more
+//                          than 8 (log2 units) above m, moves m and rescales
+//                          its row of O in TMEM; below that P stays under 2^8
+//                          and the result is the same
 //   O  += P V             tcgen05.mma, M = 128, N = D, K = 64 context rows; V
 //                          read MN-major straight from its row-major block
-// Warp 4 allocates TMEM (64 columns of S, 128 of O) and one lane issues the
-// MMAs; every thread loads context blocks (cp.async, two stages) and the
-// rotated Q tile.  The softmax warps write O / l at the end.  Every mbarrier
-// wait is bounded: on timeout the CTA raises MSA_DEVERR_WAIT_TIMEOUT and skips
-// the rest (its outputs are then void), draining issued MMAs before TMEM is
-// freed.
+// Roles (warp-specialised, synchronised by mbarriers only):
+//   warps 0-3, 4-7  tile A, tile B: rotate the Q tile into shared memory, the
+//                   softmax, then O / l to global memory
+//   warp 8          owns TMEM (all 512 columns: S buffers and O of both
+//                   tiles); lane 0 issues every MMA as soon as its inputs are
+//                   ready, in whatever order they become ready
+//   warps 9-10      stream K/V blocks through a ring of kPtcStages stages with
+//                   cp.async (warp 9 also builds the chunk table, after the
+//                   first local blocks are in flight); each lane's copies of a
+//                   block arrive on the stage's barrier when they complete, and a
+//                   stage is refilled once every P V that reads it has completed
+// Every wait is bounded: on timeout the CTA raises MSA_DEVERR_WAIT_TIMEOUT,
+// every role skips the rest (the outputs are then void), and issued MMAs are
+// drained before TMEM is freed.
 #pragma once
 #include "attend.cuh"
 #include "tc05.cuh"
@@ -35,8 +49,27 @@ namespace msa {
 
 constexpr int kPtcRows = 128;             // query rows per tile (UMMA M)
 constexpr int kPtcBlk = 64;               // context rows per block (UMMA N of S, K of P V)
-constexpr int kPtcThreads = 160;          // warps 0-3 softmax / loads, warp 4 MMA
-constexpr uint32_t kPtcTmemCols = 256;    // S at [0, 64), O at [128, 256)
+constexpr int kPtcStages = 3;             // K/V ring depth
+constexpr int kPtcLoadWarps = 2;          // warps 9 .. 9 + kPtcLoadWarps - 1 stream K/V
+constexpr int kPtcThreads = 32 * (9 + kPtcLoadWarps);
+constexpr uint32_t kPtcTmemCols = 512;
+// TMEM columns: S of tile x at 128 x + 64 (u % 2) (u = the tile's block count), O of tile x
+// at 256 + 128 x
+constexpr uint32_t kPtcTmemO = 256;
+
+// mbarriers of the prefill kernel
+enum {
+  kPbFull0 = 0,                   // stage s holds its block (the copies of every loader lane) [kPtcStages]
+  kPbEmpty0 = kPtcStages,         // every P V reading stage s has completed (commit) [kPtcStages]
+  kPbS0 = 2 * kPtcStages,         // S buffer (tile x, u % 2) is computed (commit) [4]
+  kPbQ0 = kPbS0 + 4,              // tile x's rotated Q is in shared memory (128 threads) [2]
+  kPbP0 = kPbQ0 + 2,              // tile x's P is written and O rescaled (128 threads) [2]
+  kPbO0 = kPbP0 + 2,              // tile x's P V has completed (commit) [2]
+  kPbTab = kPbO0 + 2,             // the chunk table and n_mem are ready (loader lane 0)
+  kPbDrain = kPbTab + 1,          // every MMA has completed (commit)
+  kPbN = 24
+};
+static_assert(kPbDrain < kPbN, "barrier slots");
 
 template <int D>
 struct PtcSmem {
@@ -44,10 +77,10 @@ struct PtcSmem {
   static constexpr int kQBytes = kPanels * kPtcRows * 128;   // [panel][128 rows][128 B]
   static constexpr int kKVBytes = kPanels * kPtcBlk * 128;   // [panel][64 rows][128 B]
   static constexpr int kPBytes = kPtcRows * 128;             // [128 rows][64 ctx x 2 B]
-  static constexpr int kStage = 2 * kKVBytes;                // K (later P) then V
-  static_assert(kPBytes <= kKVBytes, "P takes the place of the block's K rows");
-  // Q | 2 stages | bars (s, o, drain) + TMEM slot + flag | chunk table
-  static constexpr int kFixed = 1024 + kQBytes + 2 * kStage + 64 + (2 * kMaxTopK + 1) * 4;
+  static constexpr int kStage = 2 * kKVBytes;                // K then V
+  // Q (2 tiles) | P (2 tiles) | stages | barriers | TMEM slot, fail, n_mem | prefix + bases | table
+  static constexpr int kFixed = 1024 + 2 * kQBytes + 2 * kPBytes + kPtcStages * kStage + kPbN * 8 +
+                                16 + (2 * kMaxTopK + 1) * 4;
   static int bytes(int table_cap) { return kFixed + table_cap * 4; }
 };
 
@@ -57,10 +90,66 @@ __device__ __forceinline__ uint32_t ptc_swz(int r, int c, int rows) {
   return static_cast<uint32_t>((c >> 3) * (rows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
-// grid (B * H_kv, ceil(T * G / 128)), block kPtcThreads.  append_kernel has
-// written the call's rows to the cache before this kernel runs.
+// The chunk table of query b built by one warp (the loader): table[x] = chunk
+// row of context row x < n_mem, ranks in order; the same rows as
+// build_chunk_table.  Returns n_mem in every lane.
+__device__ __forceinline__ int build_chunk_table_warp(const int32_t *__restrict__ ids_b, int k,
+                                                      const int64_t *__restrict__ doc_chunk_off,
+                                                      int n_docs, const int32_t *__restrict__ slots_b,
+                                                      int slot_chunks, int *table, int *pre,
+                                                      int *base, int table_cap, int lane) {
+  int cnt[2] = {0, 0};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int r = lane + 32 * h;
+    if (r < k) {
+      const int d = ids_b[r];
+      if (d >= 0 && d < n_docs) {
+        const int64_t c0 = doc_chunk_off[d];
+        cnt[h] = static_cast<int>(doc_chunk_off[d + 1] - c0);
+        base[r] = slots_b ? slots_b[r] * slot_chunks : static_cast<int>(c0);
+      } else {
+        raise_device_error(MSA_DEVERR_BAD_DOC_ID);
+        base[r] = 0;
+      }
+    }
+  }
+  int run = 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    int v = cnt[h];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    const int r = lane + 32 * h;
+    const int excl = run + v - cnt[h];
+    // (a rank that would overflow the table contributes nothing; host validation keeps
+    // k * max_doc_chunks <= table_cap)
+    if (r < k) pre[r] = excl + cnt[h] > table_cap ? min(excl, table_cap) : excl;
+    run += __shfl_sync(0xffffffffu, v, 31);
+  }
+  const int n_mem = min(run, table_cap);
+  if (lane == 0) pre[k] = n_mem;
+  __syncwarp();
+  for (int x = lane; x < n_mem; x += 32) {
+    int lo = 0, hi = k - 1;  // last rank r with pre[r] <= x
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    table[x] = base[lo] + (x - pre[lo]);
+  }
+  __syncwarp();
+  return n_mem;
+}
+
+// grid (B * H_kv, ceil(ceil(T * G / 128) / 2)), block kPtcThreads, one CTA per
+// SM.  append_kernel has written the call's rows to the cache before this
+// kernel runs.
 template <int D, int G>
-__global__ void __launch_bounds__(kPtcThreads, 2)
+__global__ void __launch_bounds__(kPtcThreads, 1)
 attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
                          const int32_t *__restrict__ ids, int k,
                          const int64_t *__restrict__ doc_chunk_off, int n_docs,
@@ -74,180 +163,315 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
   static_assert(D == 128, "the tensor-core prefill takes head_dim 128");
   static_assert(G >= 1 && G <= 16 && kPtcRows % G == 0, "GQA group");
   using Sm = PtcSmem<D>;
-  constexpr int CPR = D / 8;        // 16-byte chunks per row
   constexpr int TT = kPtcRows / G;  // tokens per tile
+  constexpr int NS = kPtcStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *qs = sm;
-  uint8_t *stage0 = qs + Sm::kQBytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(stage0 + 2 * Sm::kStage);  // s, o, drain
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3);
+  uint8_t *qs0 = sm;                                   // Q of tile x at qs0 + x * kQBytes
+  uint8_t *ps0 = qs0 + 2 * Sm::kQBytes;                // P of tile x at ps0 + x * kPBytes
+  uint8_t *stage0 = ps0 + 2 * Sm::kPBytes;             // stage s at stage0 + s * kStage
+  uint64_t *bars = reinterpret_cast<uint64_t *>(stage0 + NS * Sm::kStage);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kPbN);
   volatile int *fail = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  int *pre = reinterpret_cast<int *>(bars + 8);
+  volatile int *n_mem_s = reinterpret_cast<volatile int *>(tmem_slot + 2);
+  int *pre = reinterpret_cast<int *>(tmem_slot + 4);
   int *base = pre + (kMaxTopK + 1);
   int *table = base + kMaxTopK;
-  const uint32_t bar_s = smem_u32(bars), bar_o = smem_u32(bars + 1), bar_drain = smem_u32(bars + 2);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
 
   const int H_q = H_kv * G;
   const int b = blockIdx.x / H_kv, g = blockIdx.x % H_kv;
-  const int t0 = blockIdx.y * TT;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t kv = static_cast<int64_t>(H_kv) * D;
   const int half = D / 2;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
-    mbar_init(bar_drain, 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(bar(kPbFull0 + i), 32 * kPtcLoadWarps);
+      mbar_init(bar(kPbEmpty0 + i), 1);
+    }
+    for (int i = 0; i < 4; ++i) mbar_init(bar(kPbS0 + i), 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(kPbQ0 + x), 128);
+      mbar_init(bar(kPbP0 + x), 128);
+      mbar_init(bar(kPbO0 + x), 1);
+    }
+    mbar_init(bar(kPbTab), 1);
+    mbar_init(bar(kPbDrain), 1);
     *fail = 0;
     fence_mbar_init();
   }
-  if (warp == 4) tmem_alloc(smem_u32(tmem_slot), kPtcTmemCols);
+  if (warp == 8) tmem_alloc(smem_u32(tmem_slot), kPtcTmemCols);
   griddep_wait();
   griddep_launch();
   const int len0 = cache_len[b];
-  const int n_mem = build_chunk_table(ids + static_cast<int64_t>(b) * k, k, doc_chunk_off, n_docs,
-                                      slots ? slots + static_cast<int64_t>(b) * k : nullptr,
-                                      slot_chunks, table, pre, base, table_cap);
-  // (build_chunk_table ends with __syncthreads: the barriers and the TMEM slot are visible)
+  tc05_fence_before();
+  __syncthreads();  // barriers, the fail flag and the TMEM address are visible
   tc05_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_s = tmem, tmem_o = tmem + 128;
-  const int t_last = min(t0 + TT, T_tok) - 1;
-  const int n_loc = max(0, min(len0 + t_last + 1, cap));
-  const int n_ctx = n_mem + n_loc;
-  const int nblk = (n_ctx + kPtcBlk - 1) / kPtcBlk;
 
-  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+  // the two tiles: tokens [t0x, t0x + TT), their local rows [0, n_loc[x]), nbl[x] local blocks
+  int t0[2], n_loc[2], nbl[2];
+  bool act[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    t0[x] = (2 * blockIdx.y + x) * TT;
+    act[x] = t0[x] < T_tok;
+    const int t_last = min(t0[x] + TT, T_tok) - 1;
+    n_loc[x] = act[x] ? max(0, min(len0 + t_last + 1, cap)) : 0;
+    nbl[x] = (n_loc[x] + kPtcBlk - 1) / kPtcBlk;
+  }
+  // block j < nbL: local rows [64 j, 64 j + 64); block j >= nbL: chunk rows [64 (j - nbL), ...)
+  const int nbL = max(nbl[0], nbl[1]);
+  const int n_loc_max = max(n_loc[0], n_loc[1]);
+  // does tile x read block j (every tile reads every memory block)
+  auto uses = [&](int x, int j) { return act[x] && (j < nbl[x] || j >= nbL); };
+  // the u-th block tile x reads
+  auto blk_of = [&](int x, int u) { return u < nbl[x] ? u : u + (nbL - nbl[x]); };
+
+  // bounded wait; false (and every later wait false at once) after a timeout anywhere
+  auto wait = [&](int i, uint32_t parity) -> bool {
     if (*fail) return false;
-    if (mbar_wait(bar, parity)) return true;
+    if (mbar_wait(bar(i), parity)) return true;
     *fail = 1;
     raise_device_error(MSA_DEVERR_WAIT_TIMEOUT);
     return false;
   };
 
-  // context block j (rows j*64 ..) into stage s: K and V rows, zero past the context
-  auto issue = [&](int j, int s) {
-    uint8_t *kb = stage0 + s * Sm::kStage;
-    uint8_t *vb = kb + Sm::kKVBytes;
-    for (int idx = threadIdx.x; idx < kPtcBlk * CPR; idx += kPtcThreads) {
-      const int r = idx / CPR, c = idx % CPR;
-      const int x = j * kPtcBlk + r;
-      const bool ok = x < n_ctx;
-      const __nv_bfloat16 *ksrc = K_cache, *vsrc = V_cache;
-      if (ok) {
-        if (x < n_mem) {
-          ksrc = content + static_cast<int64_t>(table[x]) * 2 * kv + g * D;
-          vsrc = ksrc + kv;
-        } else {
-          const int64_t row = (static_cast<int64_t>(b) * cap + (x - n_mem)) * kv + g * D;
-          ksrc = K_cache + row;
-          vsrc = V_cache + row;
-        }
-      }
-      cp_async_16(smem_u32(kb + ptc_swz(r, c, kPtcBlk)), ksrc + c * 8, ok);
-      cp_async_16(smem_u32(vb + ptc_swz(r, c, kPtcBlk)), vsrc + c * 8, ok);
-    }
-    cp_async_commit();
-  };
-  if (nblk > 0) issue(0, 0);
-  if (nblk > 1) issue(1, 1);
-
-  // the tile's rotated query rows (row r = token t0 + r / G, head g * G + r % G), in 16-byte
-  // pieces: item (token, chunk c of the lower half) rotates elements [8c, 8c + 8) with
-  // [half + 8c, half + 8c + 8) of the token's G heads, one RoPE load for all of them, every
-  // load of a batch of heads issued before its stores.  Rows past the call's tokens or the
-  // cache are zero.
-  {
-    constexpr int HC = D / 16;         // 16-byte chunks in half a row
-    constexpr int GB = G < 4 ? G : 4;  // heads per batch of loads
-    for (int it = threadIdx.x; it < TT * HC; it += kPtcThreads) {
-      const int tt = it / HC, c = it % HC, t = t0 + tt;
-      const bool live = t < T_tok && len0 + t < cap;
-      float2 cs[8];
-      const __nv_bfloat16 *q0 = Q;
-      if (live) {
-        const float4 *cp = reinterpret_cast<const float4 *>(
-            rope + static_cast<int64_t>(pos_offset + len0 + t) * half + c * 8);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 v = __ldg(cp + u);
-          cs[2 * u] = make_float2(v.x, v.y);
-          cs[2 * u + 1] = make_float2(v.z, v.w);
-        }
-        q0 = Q + ((static_cast<int64_t>(b) * T_tok + t) * H_q + g * G) * D + c * 8;
-      }
-#pragma unroll
-      for (int h0 = 0; h0 < G; h0 += GB) {
-        uint4 lo[GB], hi[GB];
-#pragma unroll
-        for (int h = 0; h < GB; ++h) {
-          lo[h] = live ? __ldg(reinterpret_cast<const uint4 *>(q0 + (h0 + h) * D)) : make_uint4(0, 0, 0, 0);
-          hi[h] = live ? __ldg(reinterpret_cast<const uint4 *>(q0 + (h0 + h) * D + half))
-                       : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int h = 0; h < GB; ++h) {
-          const int r = tt * G + h0 + h;
-          const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(&lo[h]);
-          const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&hi[h]);
-          uint32_t wl[4], wh[4];
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            const float2 fa = __bfloat1622float2(a[p]), fe = __bfloat1622float2(e[p]);
-            const float2 c0 = live ? cs[2 * p] : make_float2(0.0f, 0.0f);
-            const float2 c1 = live ? cs[2 * p + 1] : make_float2(0.0f, 0.0f);
-            wl[p] = pack_bf16x2(fa.x * c0.x - fe.x * c0.y, fa.y * c1.x - fe.y * c1.y);
-            wh[p] = pack_bf16x2(fe.x * c0.x + fa.x * c0.y, fe.y * c1.x + fa.y * c1.y);
+  if (warp >= 9) {
+    // ------------------------------------------------------------ loaders
+    const int lw = warp - 9;
+    // lane: 16-byte chunk lane % 16 of rows (lane / 16) + 2 lw, then every 2 kPtcLoadWarps
+    const int c = lane & 15, r0 = (lane >> 4) + 2 * lw;
+    int n_mem = 0;
+    auto issue = [&](int j) {
+      uint8_t *kb = stage0 + (j % NS) * Sm::kStage;
+      uint8_t *vb = kb + Sm::kKVBytes;
+#pragma unroll 4
+      for (int r = r0; r < kPtcBlk; r += 2 * kPtcLoadWarps) {
+        const __nv_bfloat16 *ksrc = K_cache, *vsrc = V_cache;
+        bool ok;
+        if (j < nbL) {
+          const int l = j * kPtcBlk + r;
+          ok = l < n_loc_max;
+          const int64_t row = (static_cast<int64_t>(b) * cap + l) * kv + g * D;
+          if (ok) {
+            ksrc = K_cache + row;
+            vsrc = V_cache + row;
           }
-          *reinterpret_cast<uint4 *>(qs + ptc_swz(r, c, kPtcRows)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-          *reinterpret_cast<uint4 *>(qs + ptc_swz(r, c + HC, kPtcRows)) =
-              make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        } else {
+          const int x = (j - nbL) * kPtcBlk + r;
+          ok = x < n_mem;
+          if (ok) {
+            ksrc = content + static_cast<int64_t>(table[x]) * 2 * kv + g * D;
+            vsrc = ksrc + kv;
+          }
+        }
+        cp_async_16(smem_u32(kb + ptc_swz(r, c, kPtcBlk)), ksrc + c * 8, ok);
+        cp_async_16(smem_u32(vb + ptc_swz(r, c, kPtcBlk)), vsrc + c * 8, ok);
+      }
+      cp_async_commit();
+    };
+    // block j into stage j % NS; the lane's copies arrive on the stage's barrier once they land
+    auto issue_arrive = [&](int j) {
+      issue(j);
+      cp_async_mbar_arrive_noinc(bar(kPbFull0 + j % NS));
+    };
+    // the first local blocks go out before the chunk table is built
+    int issued = 0;
+    while (issued < min(NS, nbL)) issue_arrive(issued++);
+    if (lw == 0) {
+      n_mem = build_chunk_table_warp(ids + static_cast<int64_t>(b) * k, k, doc_chunk_off, n_docs,
+                                     slots ? slots + static_cast<int64_t>(b) * k : nullptr,
+                                     slot_chunks, table, pre, base, table_cap, lane);
+      if (lane == 0) {
+        *n_mem_s = n_mem;
+        mbar_arrive(bar(kPbTab));
+      }
+    } else {
+      n_mem = __all_sync(0xffffffffu, wait(kPbTab, 0)) ? *n_mem_s : 0;
+    }
+    const int nblk = *fail ? 0 : nbL + (n_mem + kPtcBlk - 1) / kPtcBlk;
+    while (issued < min(NS, nblk)) issue_arrive(issued++);
+    // block j >= NS refills stage j % NS once every P V reading block j - NS has completed
+    for (; issued < nblk; ++issued) {
+      if (!wait(kPbEmpty0 + issued % NS, ((issued - NS) / NS) & 1)) break;
+      issue_arrive(issued);
+    }
+    cp_async_wait<0>();
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const bool tab_ok = wait(kPbTab, 0);
+      const int n_mem = tab_ok ? *n_mem_s : 0;
+      const int nbm = (n_mem + kPtcBlk - 1) / kPtcBlk;
+      int n_u[2];
+#pragma unroll
+      for (int x = 0; x < 2; ++x) n_u[x] = (tab_ok && act[x]) ? nbl[x] + nbm : 0;
+      constexpr uint32_t idesc_s = umma_idesc_bf16_f32<kPtcRows, kPtcBlk>();
+      constexpr uint32_t idesc_o = umma_idesc_bf16_f32_bmn<kPtcRows, D>();
+      bool ok = true;
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+        if (n_u[x] > 0) ok = ok && wait(kPbQ0 + x, 0);
+      int next_s[2] = {0, 0}, next_pv[2] = {0, 0};
+      uint32_t one_done = 0;  // bit s: one of the two P V reading stage s's block was issued
+      long long t_prog = clock64();
+      while (ok && (next_pv[0] < n_u[0] || next_pv[1] < n_u[1])) {
+        bool prog = false;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          // P V of the tile's block next_pv as soon as its P is written (and O rescaled)
+          if (next_pv[x] < n_u[x] && mbar_try_wait(bar(kPbP0 + x), next_pv[x] & 1)) {
+            tc05_fence_after();
+            const int j = blk_of(x, next_pv[x]);
+            const uint32_t p_addr = smem_u32(ps0 + x * Sm::kPBytes);
+            const uint32_t v_addr = smem_u32(stage0 + (j % NS) * Sm::kStage) + Sm::kKVBytes;
+#pragma unroll
+            for (int ks = 0; ks < kPtcBlk / 16; ++ks)
+              umma_bf16(tmem + kPtcTmemO + 128 * x, umma_desc_k_sw128(p_addr + ks * 32),
+                        umma_desc_mn_sw128(v_addr + ks * 16 * 128, Sm::kKVBytes / Sm::kPanels),
+                        idesc_o, (next_pv[x] | ks) != 0);
+            umma_commit(bar(kPbO0 + x));
+            const uint32_t bit = 1u << (j % NS);
+            if (!(uses(0, j) && uses(1, j)) || (one_done & bit)) {  // the last P V reading j
+              one_done &= ~bit;
+              umma_commit(bar(kPbEmpty0 + j % NS));
+            } else {
+              one_done |= bit;
+            }
+            ++next_pv[x];
+            prog = true;
+          }
+          // Q K^T of the tile's block next_s once it has landed and its S buffer is free (the
+          // softmax has read the S two blocks back: its P is written)
+          if (next_s[x] < n_u[x] && next_s[x] - 2 < next_pv[x]) {
+            const int j = blk_of(x, next_s[x]);
+            if (mbar_try_wait(bar(kPbFull0 + j % NS), (j / NS) & 1)) {
+              // the loaders' cp.async writes (generic proxy) before the tensor cores read them
+              fence_proxy_async_smem();
+              tc05_fence_after();
+              const uint32_t q_addr = smem_u32(qs0 + x * Sm::kQBytes);
+              const uint32_t k_addr = smem_u32(stage0 + (j % NS) * Sm::kStage);
+              const uint32_t d_s = tmem + 128 * x + kPtcBlk * (next_s[x] & 1);
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t pa = static_cast<uint32_t>((kk >> 2) * kPtcRows * 128 + (kk & 3) * 32);
+                const uint32_t pb = static_cast<uint32_t>((kk >> 2) * kPtcBlk * 128 + (kk & 3) * 32);
+                umma_bf16(d_s, umma_desc_k_sw128(q_addr + pa), umma_desc_k_sw128(k_addr + pb),
+                          idesc_s, kk != 0);
+              }
+              umma_commit(bar(kPbS0 + 2 * x + (next_s[x] & 1)));
+              ++next_s[x];
+              prog = true;
+            }
+          }
+        }
+        if (prog) {
+          t_prog = clock64();
+        } else if (*fail) {
+          ok = false;
+        } else if (clock64() - t_prog > kWaitBudgetCycles) {
+          *fail = 1;
+          raise_device_error(MSA_DEVERR_WAIT_TIMEOUT);
+          ok = false;
+        }
+      }
+      // every MMA issued here completes before TMEM is freed
+      umma_commit(bar(kPbDrain));
+      mbar_wait(bar(kPbDrain), 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax, tile x
+    const int x = warp >> 2;
+    const int tid = threadIdx.x & 127;
+    uint8_t *qs = qs0 + x * Sm::kQBytes;
+    uint8_t *psm = ps0 + x * Sm::kPBytes;
+    const int tq0 = x ? t0[1] : t0[0];
+    const int nbl_x = x ? nbl[1] : nbl[0];
+    const int n_loc_x = x ? n_loc[1] : n_loc[0];
+    const bool act_x = x ? act[1] : act[0];
+    // the tile's rotated query rows (row r = token tq0 + r / G, head g * G + r % G), in
+    // 16-byte pieces: item (token, chunk c of the lower half) rotates elements [8c, 8c + 8)
+    // with [half + 8c, half + 8c + 8) of the token's G heads, one RoPE load for all of them,
+    // every load of a batch of heads issued before its stores.  Rows past the call's tokens
+    // or the cache are zero.
+    {
+      constexpr int HC = D / 16;         // 16-byte chunks in half a row
+      constexpr int GB = G < 4 ? G : 4;  // heads per batch of loads
+      for (int it = tid; it < TT * HC; it += 128) {
+        const int tt = it / HC, c = it % HC, t = tq0 + tt;
+        const bool live = t < T_tok && len0 + t < cap;
+        float2 cs[8];
+        const __nv_bfloat16 *q0 = Q;
+        if (live) {
+          const float4 *cp = reinterpret_cast<const float4 *>(
+              rope + static_cast<int64_t>(pos_offset + len0 + t) * half + c * 8);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 v = __ldg(cp + u);
+            cs[2 * u] = make_float2(v.x, v.y);
+            cs[2 * u + 1] = make_float2(v.z, v.w);
+          }
+          q0 = Q + ((static_cast<int64_t>(b) * T_tok + t) * H_q + g * G) * D + c * 8;
+        }
+#pragma unroll
+        for (int h0 = 0; h0 < G; h0 += GB) {
+          uint4 lo[GB], hi[GB];
+#pragma unroll
+          for (int h = 0; h < GB; ++h) {
+            lo[h] = live ? __ldg(reinterpret_cast<const uint4 *>(q0 + (h0 + h) * D))
+                         : make_uint4(0, 0, 0, 0);
+            hi[h] = live ? __ldg(reinterpret_cast<const uint4 *>(q0 + (h0 + h) * D + half))
+                         : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int h = 0; h < GB; ++h) {
+            const int r = tt * G + h0 + h;
+            const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(&lo[h]);
+            const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&hi[h]);
+            uint32_t wl[4], wh[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const float2 fa = __bfloat1622float2(a[p]), fe = __bfloat1622float2(e[p]);
+              const float2 c0 = live ? cs[2 * p] : make_float2(0.0f, 0.0f);
+              const float2 c1 = live ? cs[2 * p + 1] : make_float2(0.0f, 0.0f);
+              wl[p] = pack_bf16x2(fa.x * c0.x - fe.x * c0.y, fa.y * c1.x - fe.y * c1.y);
+              wh[p] = pack_bf16x2(fe.x * c0.x + fa.x * c0.y, fe.y * c1.x + fa.y * c1.y);
+            }
+            *reinterpret_cast<uint4 *>(qs + ptc_swz(r, c, kPtcRows)) =
+                make_uint4(wl[0], wl[1], wl[2], wl[3]);
+            *reinterpret_cast<uint4 *>(qs + ptc_swz(r, c + HC, kPtcRows)) =
+                make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          }
         }
       }
     }
-  }
+    fence_proxy_async_smem();  // Q becomes visible to the tensor cores
+    mbar_arrive(bar(kPbQ0 + x));
 
-  // softmax state of this thread's row (warps 0-3)
-  const int r = threadIdx.x;  // (valid for warps 0-3: the TMEM lane of the row)
-  const int t_row = t0 + r / G;
-  const int vis = n_mem + len0 + t_row;  // last visible context index of the row
-  float m_run = -INFINITY, l_run = 0.0f;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-  constexpr uint32_t idesc_s = umma_idesc_bf16_f32<kPtcRows, kPtcBlk>();
-  constexpr uint32_t idesc_o = umma_idesc_bf16_f32_bmn<kPtcRows, D>();
-
-  for (int j = 0; j < nblk; ++j) {
-    const int st = j & 1;
-    uint8_t *kb = stage0 + st * Sm::kStage;
-    uint8_t *vb = kb + Sm::kKVBytes;
-    uint8_t *psm = kb;  // P [128 rows][64 context] bf16, once S = Q K^T is computed
-    if (j + 1 < nblk) cp_async_wait<1>(); else cp_async_wait<0>();
-    fence_proxy_async_smem();  // the copies (and Q) become visible to the tensor cores
-    tc05_fence_before();
-    __syncthreads();  // (A) block j is in shared memory
-    tc05_fence_after();
-    if (warp == 4 && lane == 0 && !*fail) {
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t pa = static_cast<uint32_t>((kk >> 2) * kPtcRows * 128 + (kk & 3) * 32);
-        const uint32_t pb = static_cast<uint32_t>((kk >> 2) * kPtcBlk * 128 + (kk & 3) * 32);
-        umma_bf16(tmem_s, umma_desc_k_sw128(smem_u32(qs) + pa), umma_desc_k_sw128(smem_u32(kb) + pb),
-                  idesc_s, kk != 0);
-      }
-      umma_commit(bar_s);
-    }
-    if (warp < 4) {
-      const bool ok = wait(bar_s, j & 1);
-      const bool okw = __all_sync(0xffffffffu, ok);
+    const int r = tid;  // the row = the TMEM lane
+    const int t_row = tq0 + r / G;
+    const bool tab_ok = wait(kPbTab, 0);
+    const int n_mem = tab_ok ? *n_mem_s : 0;
+    const int n_u = (tab_ok && act_x) ? nbl_x + (n_mem + kPtcBlk - 1) / kPtcBlk : 0;
+    const int vis_loc = min(len0 + t_row, n_loc_x - 1);  // last visible local row of the row
+    float m_run = -INFINITY, l_run = 0.0f;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tmem_o = tmem + kPtcTmemO + 128 * x;
+    bool okw = tab_ok;
+    for (int u = 0; u < n_u; ++u) {
+      okw = __all_sync(0xffffffffu, okw && wait(kPbS0 + 2 * x + (u & 1), (u >> 1) & 1));
+      if (!okw) break;
       tc05_fence_after();
-      // the row's last visible context index, relative to this block (-1: nothing)
-      const int lim = okw ? min(vis, n_ctx - 1) - j * kPtcBlk : -1;
+      // the row's last visible column of this block
+      const int lim = u < nbl_x ? vis_loc - u * kPtcBlk : n_mem - 1 - (u - nbl_x) * kPtcBlk;
       float s[kPtcBlk];
       static_assert(kPtcBlk == 64, "one 64-column TMEM load per block");
-      if (okw) tmem_ld64(tmem_s + lane_base, s);
-      if (lim < kPtcBlk - 1) {  // a diagonal block (or the context's ragged end): mask
+      tmem_ld64(tmem + 128 * x + kPtcBlk * (u & 1) + lane_base, s);
+      if (lim < kPtcBlk - 1) {  // a diagonal or ragged block: mask
 #pragma unroll
         for (int i = 0; i < kPtcBlk; ++i) s[i] = i <= lim ? s[i] : -INFINITY;
       }
@@ -262,95 +486,77 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
       const float mo = m_new == -INFINITY ? 0.0f : m_new;  // masked entries give 2^-inf = 0
       float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int c = 0; c < kPtcBlk; c += 8) {
-        float pv[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          pv[i] = ex2_approx(fmaf(s[c + i], scale_log2, -mo));
-          ps[i & 3] += pv[i];
-        }
-        uint4 w;
-        w.x = pack_bf16x2(pv[0], pv[1]);
-        w.y = pack_bf16x2(pv[2], pv[3]);
-        w.z = pack_bf16x2(pv[4], pv[5]);
-        w.w = pack_bf16x2(pv[6], pv[7]);
-        // (the previous block's P V completed before this block began: P is free)
-        *reinterpret_cast<uint4 *>(psm + ptc_swz(r, c / 8, kPtcRows)) = w;
+      for (int i = 0; i < kPtcBlk; ++i) {
+        s[i] = ex2_approx(fmaf(s[i], scale_log2, -mo));
+        ps[i & 3] += s[i];
       }
-      const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      l_run = l_run * alpha + psum;
+      l_run = l_run * alpha + (ps[0] + ps[1]) + (ps[2] + ps[3]);
       m_run = m_new;
-      // O's row: rescale when the max rose (the previous block's P V has completed).  The
-      // TMEM loads and stores are warp-collective: the warp takes them when any of its rows
-      // needs it, each thread with its own factor (1 where nothing rose).
-      if (j > 0 && okw && __any_sync(0xffffffffu, alpha < 1.0f)) {
+      if (u > 0) {
+        // the tile's previous P V has completed (waited at every block, so the barrier's
+        // phases are never ambiguous): the P buffer is free, and O's row is rescaled when
+        // the max rose.  TMEM loads and stores are warp-collective: the warp takes them
+        // when any of its rows needs it, each thread with its own factor.
+        okw = __all_sync(0xffffffffu, wait(kPbO0 + x, (u - 1) & 1));
+        if (!okw) break;
+        tc05_fence_after();
+        if (__any_sync(0xffffffffu, alpha < 1.0f)) {
 #pragma unroll 1
-        for (int c = 0; c < D; c += 16) {
-          float x[16];
-          tmem_ld16(tmem_o + lane_base + c, x);
+          for (int cc = 0; cc < D; cc += 16) {
+            float o[16];
+            tmem_ld16(tmem_o + lane_base + cc, o);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) x[i] *= alpha;
-          tmem_st16(tmem_o + lane_base + c, x);
+            for (int i = 0; i < 16; ++i) o[i] *= alpha;
+            tmem_st16(tmem_o + lane_base + cc, o);
+          }
         }
+      }
+#pragma unroll
+      for (int cc = 0; cc < kPtcBlk; cc += 8) {
+        uint4 w;
+        w.x = pack_bf16x2(s[cc], s[cc + 1]);
+        w.y = pack_bf16x2(s[cc + 2], s[cc + 3]);
+        w.z = pack_bf16x2(s[cc + 4], s[cc + 5]);
+        w.w = pack_bf16x2(s[cc + 6], s[cc + 7]);
+        *reinterpret_cast<uint4 *>(psm + ptc_swz(r, cc / 8, kPtcRows)) = w;
       }
       fence_proxy_async_smem();  // P becomes visible to the tensor cores
       tc05_fence_before();
+      mbar_arrive(bar(kPbP0 + x));
     }
-    __syncthreads();  // (B) P and O are ready for this block's P V
-    tc05_fence_after();
-    if (warp == 4 && lane == 0 && !*fail) {
-#pragma unroll
-      for (int ks = 0; ks < kPtcBlk / 16; ++ks)
-        umma_bf16(tmem_o, umma_desc_k_sw128(smem_u32(psm) + ks * 32),
-                  umma_desc_mn_sw128(smem_u32(vb) + ks * 16 * 128, Sm::kKVBytes / Sm::kPanels),
-                  idesc_o, (j | ks) != 0);
-      umma_commit(bar_o);
-    }
-    // every thread: the P V of this block must finish before P and this stage are reused
-    wait(bar_o, j & 1);
-    tc05_fence_after();
-    if (j + 2 < nblk) issue(j + 2, st);
-  }
-
-  // O / l for the rows of this call's tokens (the TMEM loads by whole warps)
-  const bool row_out = warp < 4 && t_row <= t_last && t_row < T_tok;
-  const bool have_o = warp < 4 && nblk > 0 && __all_sync(0xffffffffu, !*fail);
-  if (have_o) {
-    const bool live = len0 + t_row < cap && l_run > 0.0f;
-    const float inv = live ? 1.0f / l_run : 0.0f;
+    // O / l for the rows of this call's tokens (TMEM loads by whole warps)
+    const bool row_out = act_x && t_row < min(tq0 + TT, T_tok);
+    if (okw && n_u > 0) okw = __all_sync(0xffffffffu, wait(kPbO0 + x, (n_u - 1) & 1));
     __nv_bfloat16 *orow = O + ((static_cast<int64_t>(b) * T_tok + t_row) * H_q + g * G + r % G) * D;
+    if (okw && n_u > 0) {
+      tc05_fence_after();
+      const bool live = len0 + t_row < cap && l_run > 0.0f;
+      const float inv = live ? 1.0f / l_run : 0.0f;
 #pragma unroll 1
-    for (int c = 0; c < D; c += 16) {
-      float x[16];
-      tmem_ld16(tmem_o + lane_base + c, x);
-      if (!row_out) continue;
-      uint4 w0, w1;
-      w0.x = pack_bf16x2(x[0] * inv, x[1] * inv);
-      w0.y = pack_bf16x2(x[2] * inv, x[3] * inv);
-      w0.z = pack_bf16x2(x[4] * inv, x[5] * inv);
-      w0.w = pack_bf16x2(x[6] * inv, x[7] * inv);
-      w1.x = pack_bf16x2(x[8] * inv, x[9] * inv);
-      w1.y = pack_bf16x2(x[10] * inv, x[11] * inv);
-      w1.z = pack_bf16x2(x[12] * inv, x[13] * inv);
-      w1.w = pack_bf16x2(x[14] * inv, x[15] * inv);
-      *reinterpret_cast<uint4 *>(orow + c) = w0;
-      *reinterpret_cast<uint4 *>(orow + c + 8) = w1;
+      for (int cc = 0; cc < D; cc += 16) {
+        float o[16];
+        tmem_ld16(tmem_o + lane_base + cc, o);
+        if (!row_out) continue;
+        uint4 w0, w1;
+        w0.x = pack_bf16x2(o[0] * inv, o[1] * inv);
+        w0.y = pack_bf16x2(o[2] * inv, o[3] * inv);
+        w0.z = pack_bf16x2(o[4] * inv, o[5] * inv);
+        w0.w = pack_bf16x2(o[6] * inv, o[7] * inv);
+        w1.x = pack_bf16x2(o[8] * inv, o[9] * inv);
+        w1.y = pack_bf16x2(o[10] * inv, o[11] * inv);
+        w1.z = pack_bf16x2(o[12] * inv, o[13] * inv);
+        w1.w = pack_bf16x2(o[14] * inv, o[15] * inv);
+        *reinterpret_cast<uint4 *>(orow + cc) = w0;
+        *reinterpret_cast<uint4 *>(orow + cc + 8) = w1;
+      }
+    } else if (row_out) {
+      for (int cc = 0; cc < D; cc += 8) *reinterpret_cast<uint4 *>(orow + cc) = make_uint4(0, 0, 0, 0);
     }
-  } else if (row_out) {
-    __nv_bfloat16 *orow = O + ((static_cast<int64_t>(b) * T_tok + t_row) * H_q + g * G + r % G) * D;
-    for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4 *>(orow + c) = make_uint4(0, 0, 0, 0);
   }
   tc05_fence_before();
   __syncthreads();
   tc05_fence_after();
-  if (warp == 4) {
-    if (lane == 0) {  // every MMA issued here has completed before TMEM is freed
-      umma_commit(bar_drain);
-      mbar_wait(bar_drain, 0);
-    }
-    __syncwarp();
-    tmem_dealloc(tmem, kPtcTmemCols);
-  }
+  if (warp == 8) tmem_dealloc(tmem, kPtcTmemCols);
 }
 
 }  // namespace msa

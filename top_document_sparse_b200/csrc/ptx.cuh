@@ -128,6 +128,12 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, bool 
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n)
                : "memory");
 }
+// Arrive on `bar` once every cp.async this thread has issued so far has
+// completed; the arrival counts toward the barrier's expected count (.noinc).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
