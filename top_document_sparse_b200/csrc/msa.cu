@@ -183,6 +183,24 @@ msa_status make_map_bf16(CUtensorMap *map, const void *base, int64_t rows, int64
   return MSA_OK;
 }
 
+// 3-D bf16 map over [d2][d1][d0] with the given byte strides of dimensions 1 and 2, box
+// {64, box1, box2}, 128-byte swizzle, out-of-range elements read as zero.
+msa_status make_map_bf16_3d(CUtensorMap *map, const void *base, int64_t d0, int64_t d1, int64_t d2,
+                            int64_t stride1, int64_t stride2, int box1, int box2) {
+  auto fn = encode_tiled();
+  if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d0), static_cast<cuuint64_t>(d1),
+                        static_cast<cuuint64_t>(d2)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(stride1), static_cast<cuuint64_t>(stride2)};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box1), static_cast<cuuint32_t>(box2)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MSA_OK;
+}
+
 // ---------------------------------------------------------------- helpers
 size_t elem_size(msa_dtype t) { return t == MSA_BF16 ? 2 : 4; }
 
@@ -368,6 +386,15 @@ msa_status launch_attend_mma(const msa_memory *mem, const void *content, const i
     if (T > 1 && smem_pt <= max_dyn_smem()) {
       // several tokens (prefill), tensor cores: one CTA per (query, kv head, pair of adjacent
       // tiles of 128 / G tokens x G heads); append_kernel ran before
+      // the local cache as [B * cap rows][H_kv][D]: box {64 of D, head g, 64 rows}
+      CUtensorMap tm_k, tm_v;
+      const int64_t row_bytes = static_cast<int64_t>(mem->H_kv) * D * 2;
+      msa_status ms = make_map_bf16_3d(&tm_k, Kc, D, mem->H_kv, static_cast<int64_t>(B) * cap,
+                                       D * 2, row_bytes, 1, msa::kPtcBlk);
+      if (ms != MSA_OK) return ms;
+      ms = make_map_bf16_3d(&tm_v, Vc, D, mem->H_kv, static_cast<int64_t>(B) * cap, D * 2,
+                            row_bytes, 1, msa::kPtcBlk);
+      if (ms != MSA_OK) return ms;
       auto kpt = msa::attend_prefill_tc_kernel<128, G>;
       MSA_CUDA(cudaFuncSetAttribute(kpt, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_pt));
       constexpr int TT = msa::kPtcRows / G;
@@ -382,7 +409,7 @@ msa_status launch_attend_mma(const msa_memory *mem, const void *content, const i
                           static_cast<const __nv_bfloat16 *>(Vc),
                           static_cast<const int32_t *>(cache_len), cap, pos_offset,
                           static_cast<const float2 *>(mem->d_rope), scale_log2, plan.table_cap,
-                          static_cast<__nv_bfloat16 *>(O)));
+                          static_cast<__nv_bfloat16 *>(O), tm_k, tm_v));
       MSA_LAUNCHED("attend_prefill_tc_kernel");
       MSA_CUDA(launch_pdl(msa::advance_kernel, dim3((B + 255) / 256), dim3(256), 0, st, cache_len,
                           B, T, cap));

@@ -33,11 +33,15 @@
 //   warp 8          owns TMEM (all 512 columns: S buffers and O of both
 //                   tiles); lane 0 issues every MMA as soon as its inputs are
 //                   ready, in whatever order they become ready
-//   warps 9-10      stream K/V blocks through a ring of kPtcStages stages with
-//                   cp.async (warp 9 also builds the chunk table, after the
-//                   first local blocks are in flight); each lane's copies of a
-//                   block arrive on the stage's barrier when they complete, and a
-//                   stage is refilled once every P V that reads it has completed
+//   warps 9-10      stream K/V blocks through a ring of kPtcStages stages:
+//                   whole local blocks by TMA (one thread), the ragged last
+//                   local block and the retrieved chunks (through the chunk
+//                   table, which warp 9 builds after the first local blocks are
+//                   in flight) by cp.async, each lane's copies arriving on the
+//                   stage's barrier when they complete; a stage is refilled once
+//                   every P V that reads it has completed.  The softmax and the
+//                   MMA issuer take the local blocks before they wait for the
+//                   table.
 // Every wait is bounded: on timeout the CTA raises MSA_DEVERR_WAIT_TIMEOUT,
 // every role skips the rest (the outputs are then void), and issued MMAs are
 // drained before TMEM is freed.
@@ -147,7 +151,9 @@ __device__ __forceinline__ int build_chunk_table_warp(const int32_t *__restrict_
 
 // grid (B * H_kv, ceil(ceil(T * G / 128) / 2)), block kPtcThreads, one CTA per
 // SM.  append_kernel has written the call's rows to the cache before this
-// kernel runs.
+// kernel runs.  tm_k / tm_v map the local cache as [B * cap rows][H_kv][D]
+// with box {64 of D, 1 head, 64 rows} (128-byte swizzle): a whole local block
+// of the CTA's kv head is two TMA loads per tensor.
 template <int D, int G>
 __global__ void __launch_bounds__(kPtcThreads, 1)
 attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
@@ -159,7 +165,8 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
                          const __nv_bfloat16 *__restrict__ V_cache,
                          const int32_t *__restrict__ cache_len, int cap, int pos_offset,
                          const float2 *__restrict__ rope, float scale_log2, int table_cap,
-                         __nv_bfloat16 *__restrict__ O) {
+                         __nv_bfloat16 *__restrict__ O, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v) {
   static_assert(D == 128, "the tensor-core prefill takes head_dim 128");
   static_assert(G >= 1 && G <= 16 && kPtcRows % G == 0, "GQA group");
   using Sm = PtcSmem<D>;
@@ -273,10 +280,27 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
       }
       cp_async_commit();
     };
-    // block j into stage j % NS; the lane's copies arrive on the stage's barrier once they land
+    // block j into stage j % NS: a whole local block by TMA (every other loader lane arrives
+    // at once), otherwise each lane's copies arrive on the stage's barrier once they land
     auto issue_arrive = [&](int j) {
-      issue(j);
-      cp_async_mbar_arrive_noinc(bar(kPbFull0 + j % NS));
+      const uint32_t fb = bar(kPbFull0 + j % NS);
+      if (j < nbL && (j + 1) * kPtcBlk <= n_loc_max) {
+        if (lw == 0 && lane == 0) {
+          mbar_arrive_expect_tx(fb, static_cast<uint32_t>(Sm::kStage));
+          const uint32_t kb = smem_u32(stage0 + (j % NS) * Sm::kStage);
+          const int row = b * cap + j * kPtcBlk;
+#pragma unroll
+          for (int p = 0; p < Sm::kPanels; ++p) {
+            tma_load_3d(kb + p * (kPtcBlk * 128), &tm_k, 64 * p, g, row, fb);
+            tma_load_3d(kb + Sm::kKVBytes + p * (kPtcBlk * 128), &tm_v, 64 * p, g, row, fb);
+          }
+        } else {
+          mbar_arrive(fb);
+        }
+      } else {
+        issue(j);
+        cp_async_mbar_arrive_noinc(fb);
+      }
     };
     // the first local blocks go out before the chunk table is built
     int issued = 0;
@@ -303,27 +327,31 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const bool tab_ok = wait(kPbTab, 0);
-      const int n_mem = tab_ok ? *n_mem_s : 0;
-      const int nbm = (n_mem + kPtcBlk - 1) / kPtcBlk;
-      int n_u[2];
-#pragma unroll
-      for (int x = 0; x < 2; ++x) n_u[x] = (tab_ok && act[x]) ? nbl[x] + nbm : 0;
+      // until the chunk table is known, only the local blocks
+      int n_u[2] = {act[0] ? nbl[0] : 0, act[1] ? nbl[1] : 0};
+      bool have_tab = false;
       constexpr uint32_t idesc_s = umma_idesc_bf16_f32<kPtcRows, kPtcBlk>();
       constexpr uint32_t idesc_o = umma_idesc_bf16_f32_bmn<kPtcRows, D>();
       bool ok = true;
 #pragma unroll
       for (int x = 0; x < 2; ++x)
-        if (n_u[x] > 0) ok = ok && wait(kPbQ0 + x, 0);
+        if (act[x]) ok = ok && wait(kPbQ0 + x, 0);
       int next_s[2] = {0, 0}, next_pv[2] = {0, 0};
       uint32_t one_done = 0;  // bit s: one of the two P V reading stage s's block was issued
       long long t_prog = clock64();
-      while (ok && (next_pv[0] < n_u[0] || next_pv[1] < n_u[1])) {
+      while (ok && (!have_tab || next_pv[0] < n_u[0] || next_pv[1] < n_u[1])) {
         bool prog = false;
+        if (!have_tab && mbar_test_wait(bar(kPbTab), 0)) {
+          have_tab = true;
+          const int nbm = (*n_mem_s + kPtcBlk - 1) / kPtcBlk;
+#pragma unroll
+          for (int x = 0; x < 2; ++x) n_u[x] = act[x] ? nbl[x] + nbm : 0;
+          prog = true;
+        }
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
           // P V of the tile's block next_pv as soon as its P is written (and O rescaled)
-          if (next_pv[x] < n_u[x] && mbar_try_wait(bar(kPbP0 + x), next_pv[x] & 1)) {
+          if (next_pv[x] < n_u[x] && mbar_test_wait(bar(kPbP0 + x), next_pv[x] & 1)) {
             tc05_fence_after();
             const int j = blk_of(x, next_pv[x]);
             const uint32_t p_addr = smem_u32(ps0 + x * Sm::kPBytes);
@@ -348,7 +376,7 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
           // softmax has read the S two blocks back: its P is written)
           if (next_s[x] < n_u[x] && next_s[x] - 2 < next_pv[x]) {
             const int j = blk_of(x, next_s[x]);
-            if (mbar_try_wait(bar(kPbFull0 + j % NS), (j / NS) & 1)) {
+            if (mbar_test_wait(bar(kPbFull0 + j % NS), (j / NS) & 1)) {
               // the loaders' cp.async writes (generic proxy) before the tensor cores read them
               fence_proxy_async_smem();
               tc05_fence_after();
@@ -454,16 +482,24 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
 
     const int r = tid;  // the row = the TMEM lane
     const int t_row = tq0 + r / G;
-    const bool tab_ok = wait(kPbTab, 0);
-    const int n_mem = tab_ok ? *n_mem_s : 0;
-    const int n_u = (tab_ok && act_x) ? nbl_x + (n_mem + kPtcBlk - 1) / kPtcBlk : 0;
+    // the local blocks first; the chunk table (n_mem) only when they are done
+    int n_u = act_x ? nbl_x : 0, n_mem = 0;
+    bool have_tab = false;
     const int vis_loc = min(len0 + t_row, n_loc_x - 1);  // last visible local row of the row
     float m_run = -INFINITY, l_run = 0.0f;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tmem_o = tmem + kPtcTmemO + 128 * x;
-    bool okw = tab_ok;
-    for (int u = 0; u < n_u; ++u) {
-      okw = __all_sync(0xffffffffu, okw && wait(kPbS0 + 2 * x + (u & 1), (u >> 1) & 1));
+    bool okw = true;
+    for (int u = 0;; ++u) {
+      if (u >= n_u && !have_tab) {
+        have_tab = true;
+        okw = __all_sync(0xffffffffu, wait(kPbTab, 0));
+        if (!okw) break;
+        n_mem = *n_mem_s;
+        n_u = act_x ? nbl_x + (n_mem + kPtcBlk - 1) / kPtcBlk : 0;
+      }
+      if (u >= n_u) break;
+      okw = __all_sync(0xffffffffu, wait(kPbS0 + 2 * x + (u & 1), (u >> 1) & 1));
       if (!okw) break;
       tc05_fence_after();
       // the row's last visible column of this block
