@@ -373,6 +373,48 @@ msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, i
   return launch_topk<64>(mem, state, exclude, B, k, plan.n_split, cand, ids, scores, st);
 }
 
+// The tensor-core prefill (head_dim 128, bf16) with a K/V ring of NS stages.
+template <int G, int NS>
+msa_status launch_prefill_tc(const msa_memory *mem, const void *content, const int32_t *ids,
+                             const int32_t *slots, int slot_chunks, int B, int k, int T,
+                             const void *Q, void *Kc, void *Vc, int32_t *cache_len, int cap,
+                             int pos_offset, float scale_log2, const AttendPlan &plan, void *O,
+                             cudaStream_t st) {
+  constexpr int D = 128;
+  const int smem_pt = msa::PtcSmem<D, NS>::bytes(plan.table_cap);
+  // the local cache as [B * cap rows][H_kv][D]: box {64 of D, head g, 64 rows}
+  CUtensorMap tm_k, tm_v;
+  const int64_t row_bytes = static_cast<int64_t>(mem->H_kv) * D * 2;
+  msa_status ms = make_map_bf16_3d(&tm_k, Kc, D, mem->H_kv, static_cast<int64_t>(B) * cap,
+                                   D * 2, row_bytes, 1, msa::kPtcBlk);
+  if (ms != MSA_OK) return ms;
+  ms = make_map_bf16_3d(&tm_v, Vc, D, mem->H_kv, static_cast<int64_t>(B) * cap, D * 2,
+                        row_bytes, 1, msa::kPtcBlk);
+  if (ms != MSA_OK) return ms;
+  auto kpt = msa::attend_prefill_tc_kernel<128, G, NS>;
+  MSA_CUDA(cudaFuncSetAttribute(kpt, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_pt));
+  constexpr int TT = msa::kPtcRows / G;
+  const int n_tiles = (T + TT - 1) / TT;
+  const int n_pairs = (n_tiles + 1) / 2;
+  const int64_t n_ctas = static_cast<int64_t>(n_pairs) * B * mem->H_kv;
+  if (n_ctas > 0x7FFFFFFF) return fail(MSA_ERR_UNSUPPORTED, "too many query tokens");
+  dim3 grid_pt(static_cast<unsigned>(n_ctas));
+  MSA_CUDA(launch_pdl(kpt, grid_pt, dim3(msa::kPtcThreads), smem_pt, st,
+                      static_cast<const __nv_bfloat16 *>(content), ids, k,
+                      static_cast<const int64_t *>(mem->d_doc_chunk_off), mem->n_docs, slots,
+                      slot_chunks, mem->H_kv, static_cast<const __nv_bfloat16 *>(Q), T,
+                      static_cast<const __nv_bfloat16 *>(Kc),
+                      static_cast<const __nv_bfloat16 *>(Vc),
+                      static_cast<const int32_t *>(cache_len), cap, pos_offset,
+                      static_cast<const float2 *>(mem->d_rope), scale_log2, plan.table_cap,
+                      static_cast<__nv_bfloat16 *>(O), tm_k, tm_v, n_pairs));
+  MSA_LAUNCHED("attend_prefill_tc_kernel");
+  MSA_CUDA(launch_pdl(msa::advance_kernel, dim3((B + 255) / 256), dim3(256), 0, st, cache_len,
+                      B, T, cap));
+  MSA_LAUNCHED("advance_kernel");
+  return MSA_OK;
+}
+
 template <int D, int G>
 msa_status launch_attend_mma(const msa_memory *mem, const void *content, const int32_t *ids,
                              const int32_t *slots, int slot_chunks, int B, int k, int T,
@@ -381,40 +423,13 @@ msa_status launch_attend_mma(const msa_memory *mem, const void *content, const i
                              const AttendPlan &plan, void *O, void *ws, cudaStream_t st) {
   const float scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)) * 1.4426950408889634);
   if constexpr (D == 128) {
-    using Pt = msa::PtcSmem<D>;
-    const int smem_pt = Pt::bytes(plan.table_cap);
-    if (T > 1 && smem_pt <= max_dyn_smem()) {
-      // several tokens (prefill), tensor cores: one CTA per (query, kv head, pair of adjacent
-      // tiles of 128 / G tokens x G heads); append_kernel ran before
-      // the local cache as [B * cap rows][H_kv][D]: box {64 of D, head g, 64 rows}
-      CUtensorMap tm_k, tm_v;
-      const int64_t row_bytes = static_cast<int64_t>(mem->H_kv) * D * 2;
-      msa_status ms = make_map_bf16_3d(&tm_k, Kc, D, mem->H_kv, static_cast<int64_t>(B) * cap,
-                                       D * 2, row_bytes, 1, msa::kPtcBlk);
-      if (ms != MSA_OK) return ms;
-      ms = make_map_bf16_3d(&tm_v, Vc, D, mem->H_kv, static_cast<int64_t>(B) * cap, D * 2,
-                            row_bytes, 1, msa::kPtcBlk);
-      if (ms != MSA_OK) return ms;
-      auto kpt = msa::attend_prefill_tc_kernel<128, G>;
-      MSA_CUDA(cudaFuncSetAttribute(kpt, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_pt));
-      constexpr int TT = msa::kPtcRows / G;
-      const int n_tiles = (T + TT - 1) / TT;
-      dim3 grid_pt(static_cast<unsigned>(B * mem->H_kv), static_cast<unsigned>((n_tiles + 1) / 2));
-      if (grid_pt.y > 65535) return fail(MSA_ERR_UNSUPPORTED, "too many query tokens");
-      MSA_CUDA(launch_pdl(kpt, grid_pt, dim3(msa::kPtcThreads), smem_pt, st,
-                          static_cast<const __nv_bfloat16 *>(content), ids, k,
-                          static_cast<const int64_t *>(mem->d_doc_chunk_off), mem->n_docs, slots,
-                          slot_chunks, mem->H_kv, static_cast<const __nv_bfloat16 *>(Q), T,
-                          static_cast<const __nv_bfloat16 *>(Kc),
-                          static_cast<const __nv_bfloat16 *>(Vc),
-                          static_cast<const int32_t *>(cache_len), cap, pos_offset,
-                          static_cast<const float2 *>(mem->d_rope), scale_log2, plan.table_cap,
-                          static_cast<__nv_bfloat16 *>(O), tm_k, tm_v));
-      MSA_LAUNCHED("attend_prefill_tc_kernel");
-      MSA_CUDA(launch_pdl(msa::advance_kernel, dim3((B + 255) / 256), dim3(256), 0, st, cache_len,
-                          B, T, cap));
-      MSA_LAUNCHED("advance_kernel");
-      return MSA_OK;
+    // several tokens (prefill), tensor cores: one CTA per (query, kv head, pair of adjacent
+    // tiles of 128 / G tokens x G heads), a K/V ring of three stages (four measured slower:
+    // 265 against 247 us at the 1M prefill); append_kernel ran before
+    if (T > 1) {
+      if (msa::PtcSmem<D, 3>::bytes(plan.table_cap) <= max_dyn_smem())
+        return launch_prefill_tc<G, 3>(mem, content, ids, slots, slot_chunks, B, k, T, Q, Kc, Vc,
+                                       cache_len, cap, pos_offset, scale_log2, plan, O, st);
     }
   }
   if (T > 1) {

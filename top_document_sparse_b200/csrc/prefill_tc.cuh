@@ -33,7 +33,7 @@
 //   warp 8          owns TMEM (all 512 columns: S buffers and O of both
 //                   tiles); lane 0 issues every MMA as soon as its inputs are
 //                   ready, in whatever order they become ready
-//   warps 9-10      stream K/V blocks through a ring of kPtcStages stages:
+//   warps 9-10      stream K/V blocks through a ring of NS stages:
 //                   whole local blocks by TMA (one thread), the ragged last
 //                   local block and the retrieved chunks (through the chunk
 //                   table, which warp 9 builds after the first local blocks are
@@ -53,7 +53,7 @@ namespace msa {
 
 constexpr int kPtcRows = 128;             // query rows per tile (UMMA M)
 constexpr int kPtcBlk = 64;               // context rows per block (UMMA N of S, K of P V)
-constexpr int kPtcStages = 3;             // K/V ring depth
+constexpr int kPtcMaxStages = 4;          // largest K/V ring depth the barriers provide for
 constexpr int kPtcLoadWarps = 2;          // warps 9 .. 9 + kPtcLoadWarps - 1 stream K/V
 constexpr int kPtcThreads = 32 * (9 + kPtcLoadWarps);
 constexpr uint32_t kPtcTmemCols = 512;
@@ -63,9 +63,9 @@ constexpr uint32_t kPtcTmemO = 256;
 
 // mbarriers of the prefill kernel
 enum {
-  kPbFull0 = 0,                   // stage s holds its block (the copies of every loader lane) [kPtcStages]
-  kPbEmpty0 = kPtcStages,         // every P V reading stage s has completed (commit) [kPtcStages]
-  kPbS0 = 2 * kPtcStages,         // S buffer (tile x, u % 2) is computed (commit) [4]
+  kPbFull0 = 0,                      // stage s holds its block (the copies of every loader lane)
+  kPbEmpty0 = kPtcMaxStages,         // every P V reading stage s has completed (commit)
+  kPbS0 = 2 * kPtcMaxStages,         // S buffer (tile x, u % 2) is computed (commit) [4]
   kPbQ0 = kPbS0 + 4,              // tile x's rotated Q is in shared memory (128 threads) [2]
   kPbP0 = kPbQ0 + 2,              // tile x's P is written and O rescaled (128 threads) [2]
   kPbO0 = kPbP0 + 2,              // tile x's P V has completed (commit) [2]
@@ -75,15 +75,16 @@ enum {
 };
 static_assert(kPbDrain < kPbN, "barrier slots");
 
-template <int D>
+template <int D, int NS>
 struct PtcSmem {
+  static_assert(NS >= 2 && NS <= kPtcMaxStages, "ring depth");
   static constexpr int kPanels = D / 64;
   static constexpr int kQBytes = kPanels * kPtcRows * 128;   // [panel][128 rows][128 B]
   static constexpr int kKVBytes = kPanels * kPtcBlk * 128;   // [panel][64 rows][128 B]
   static constexpr int kPBytes = kPtcRows * 128;             // [128 rows][64 ctx x 2 B]
   static constexpr int kStage = 2 * kKVBytes;                // K then V
   // Q (2 tiles) | P (2 tiles) | stages | barriers | TMEM slot, fail, n_mem | prefix + bases | table
-  static constexpr int kFixed = 1024 + 2 * kQBytes + 2 * kPBytes + kPtcStages * kStage + kPbN * 8 +
+  static constexpr int kFixed = 1024 + 2 * kQBytes + 2 * kPBytes + NS * kStage + kPbN * 8 +
                                 16 + (2 * kMaxTopK + 1) * 4;
   static int bytes(int table_cap) { return kFixed + table_cap * 4; }
 };
@@ -149,12 +150,14 @@ __device__ __forceinline__ int build_chunk_table_warp(const int32_t *__restrict_
   return n_mem;
 }
 
-// grid (B * H_kv, ceil(ceil(T * G / 128) / 2)), block kPtcThreads, one CTA per
-// SM.  append_kernel has written the call's rows to the cache before this
+// grid n_pairs * B * H_kv (n_pairs = ceil(ceil(T * G / 128) / 2)), block
+// kPtcThreads, one CTA per SM: the tile pairs of one (query, kv head) are
+// adjacent in launch order, so they run at about the same time and read the
+// shared context from L2, the pair with the most context first.  append_kernel has written the call's rows to the cache before this
 // kernel runs.  tm_k / tm_v map the local cache as [B * cap rows][H_kv][D]
 // with box {64 of D, 1 head, 64 rows} (128-byte swizzle): a whole local block
 // of the CTA's kv head is two TMA loads per tensor.
-template <int D, int G>
+template <int D, int G, int NS>
 __global__ void __launch_bounds__(kPtcThreads, 1)
 attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
                          const int32_t *__restrict__ ids, int k,
@@ -166,12 +169,11 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
                          const int32_t *__restrict__ cache_len, int cap, int pos_offset,
                          const float2 *__restrict__ rope, float scale_log2, int table_cap,
                          __nv_bfloat16 *__restrict__ O, const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v) {
+                         const __grid_constant__ CUtensorMap tm_v, int n_pairs) {
   static_assert(D == 128, "the tensor-core prefill takes head_dim 128");
   static_assert(G >= 1 && G <= 16 && kPtcRows % G == 0, "GQA group");
-  using Sm = PtcSmem<D>;
+  using Sm = PtcSmem<D, NS>;
   constexpr int TT = kPtcRows / G;  // tokens per tile
-  constexpr int NS = kPtcStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -188,7 +190,9 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
   auto bar = [&](int i) { return smem_u32(bars + i); };
 
   const int H_q = H_kv * G;
-  const int b = blockIdx.x / H_kv, g = blockIdx.x % H_kv;
+  const int bg = static_cast<int>(blockIdx.x / n_pairs);
+  const int b = bg / H_kv, g = bg % H_kv;
+  const int pair = n_pairs - 1 - static_cast<int>(blockIdx.x % n_pairs);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t kv = static_cast<int64_t>(H_kv) * D;
   const int half = D / 2;
@@ -210,6 +214,10 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
     fence_mbar_init();
   }
   if (warp == 8) tmem_alloc(smem_u32(tmem_slot), kPtcTmemCols);
+  if (warp == 9 && lane == 0) {
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
   griddep_wait();
   griddep_launch();
   const int len0 = cache_len[b];
@@ -223,7 +231,7 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
   bool act[2];
 #pragma unroll
   for (int x = 0; x < 2; ++x) {
-    t0[x] = (2 * blockIdx.y + x) * TT;
+    t0[x] = (2 * pair + x) * TT;
     act[x] = t0[x] < T_tok;
     const int t_last = min(t0[x] + TT, T_tok) - 1;
     n_loc[x] = act[x] ? max(0, min(len0 + t_last + 1, cap)) : 0;
@@ -289,10 +297,12 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
           mbar_arrive_expect_tx(fb, static_cast<uint32_t>(Sm::kStage));
           const uint32_t kb = smem_u32(stage0 + (j % NS) * Sm::kStage);
           const int row = b * cap + j * kPtcBlk;
+          const uint64_t keep = policy_evict_last();  // the other tiles of (b, g) read it too
 #pragma unroll
           for (int p = 0; p < Sm::kPanels; ++p) {
-            tma_load_3d(kb + p * (kPtcBlk * 128), &tm_k, 64 * p, g, row, fb);
-            tma_load_3d(kb + Sm::kKVBytes + p * (kPtcBlk * 128), &tm_v, 64 * p, g, row, fb);
+            tma_load_3d_hint(kb + p * (kPtcBlk * 128), &tm_k, 64 * p, g, row, fb, keep);
+            tma_load_3d_hint(kb + Sm::kKVBytes + p * (kPtcBlk * 128), &tm_v, 64 * p, g, row, fb,
+                             keep);
           }
         } else {
           mbar_arrive(fb);
@@ -429,6 +439,7 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
     {
       constexpr int HC = D / 16;         // 16-byte chunks in half a row
       constexpr int GB = G < 4 ? G : 4;  // heads per batch of loads
+      const uint64_t stream = policy_evict_first();  // Q is read once: keep the cache in L2
       for (int it = tid; it < TT * HC; it += 128) {
         const int tt = it / HC, c = it % HC, t = tq0 + tt;
         const bool live = t < T_tok && len0 + t < cap;
@@ -450,10 +461,8 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
           uint4 lo[GB], hi[GB];
 #pragma unroll
           for (int h = 0; h < GB; ++h) {
-            lo[h] = live ? __ldg(reinterpret_cast<const uint4 *>(q0 + (h0 + h) * D))
-                         : make_uint4(0, 0, 0, 0);
-            hi[h] = live ? __ldg(reinterpret_cast<const uint4 *>(q0 + (h0 + h) * D + half))
-                         : make_uint4(0, 0, 0, 0);
+            lo[h] = live ? ld_nc_v4_hint(q0 + (h0 + h) * D, stream) : make_uint4(0, 0, 0, 0);
+            hi[h] = live ? ld_nc_v4_hint(q0 + (h0 + h) * D + half, stream) : make_uint4(0, 0, 0, 0);
           }
 #pragma unroll
           for (int h = 0; h < GB; ++h) {
@@ -568,6 +577,7 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
       tc05_fence_after();
       const bool live = len0 + t_row < cap && l_run > 0.0f;
       const float inv = live ? 1.0f / l_run : 0.0f;
+      const uint64_t stream = policy_evict_first();  // O is not read here again
 #pragma unroll 1
       for (int cc = 0; cc < D; cc += 16) {
         float o[16];
@@ -582,8 +592,8 @@ attend_prefill_tc_kernel(const __nv_bfloat16 *__restrict__ content,
         w1.y = pack_bf16x2(o[10] * inv, o[11] * inv);
         w1.z = pack_bf16x2(o[12] * inv, o[13] * inv);
         w1.w = pack_bf16x2(o[14] * inv, o[15] * inv);
-        *reinterpret_cast<uint4 *>(orow + cc) = w0;
-        *reinterpret_cast<uint4 *>(orow + cc + 8) = w1;
+        st_v4_hint(orow + cc, w0, stream);
+        st_v4_hint(orow + cc + 8, w1, stream);
       }
     } else if (row_out) {
       for (int cc = 0; cc < D; cc += 8) *reinterpret_cast<uint4 *>(orow + cc) = make_uint4(0, 0, 0, 0);
