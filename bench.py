@@ -222,6 +222,13 @@ def prefill(mem, w, layers, msa):
     torch.cuda.synchronize()
     for L in layers:
         L.state0 = L.dec.state.clone()
+        # the attention's algorithmic work: QK^T and PV over every visible (query head, token,
+        # context row), 2 x 2 x D FLOP each; token t sees the retrieved chunk rows and local
+        # rows 0..t of this call
+        off = mem.doc_chunk_offsets
+        n_mem = np.array([sum(int(off[d + 1] - off[d]) for d in row)
+                          for row in L.dec.ids.cpu().numpy()], dtype=np.float64)
+        L.prefill_flop = 4.0 * w.head_dim * H_q * float(np.sum(n_mem * T + T * (T + 1) / 2))
         del L.prefill, L.Qr_pre
     return ev
 
@@ -501,6 +508,8 @@ def run_gpu(args, w, world, rank, local):
                           "frac": round(ceiling_ms / ms_per_step, 4)},
         "encode": {"gbs": round(enc_bytes / (enc_ms * 1e-3) / 1e9, 1), "ms": round(enc_ms, 2)},
         "prefill": {"route_ms": round(pre_route_ms, 3), "attend_ms": round(pre_attn_ms, 3),
+                    "attend_tflops": round(sum(L.prefill_flop for L in layers)
+                                           / (pre_attn_ms * 1e-3) / 1e12, 1),
                     "route_tflops": round(n_layers * 2 * B * w.query_tokens * mem.n_chunks * W_r
                                           / (pre_route_ms * 1e-3) / 1e12, 1)},
         "planted_retrieved": planted_ok,
