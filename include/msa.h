@@ -167,7 +167,11 @@ MSA_API size_t msa_route_workspace_size(const msa_memory *mem, int32_t batch,
  *                exclude[b,d] != 0; scores[b,:] their states.
  *   router_keys : device [C][H_r][d_r] as written by msa_encode_memory
  *   Qr          : device [batch][tokens][H_r][d_r]; tokens may be 0 (top-k
- *                 of the state only)
+ *                 of the state only).  Read as soon as the call's first
+ *                 kernel starts, which can be before the previous kernel of
+ *                 this library on the stream has completed (programmatic
+ *                 dependent launch): Qr must not be an output of the
+ *                 previous msa_* call on the same stream
  *   state       : device [batch][n_docs] fp32, read and updated (the running
  *                 max over every token routed so far; reset with -inf)
  *   exclude     : device [batch][n_docs] uint8 or NULL
@@ -279,6 +283,8 @@ MSA_API size_t msa_step_workspace_size(const msa_memory *mem, int32_t batch, int
  * top-k, then attend with the new token appended to the local cache.
  *   Qr_tok : device [batch][H_r][d_r];  Q_tok : [batch][n_q_heads][D]
  *   K_tok, V_tok : [batch][H_kv][D];     O_tok : [batch][n_q_heads][D]
+ * Qr_tok is read early, as msa_route's Qr: it must not be an output of the
+ * previous msa_* call on the same stream.
  */
 MSA_API msa_status msa_step(const msa_memory *mem, const void *router_keys,
                     const void *content, const msa_decode_state *st,

@@ -265,6 +265,13 @@ ATTN_CASES = [
     ("bf16", 64, 16, 16, 7, 1, 3),
     ("bf16", 128, 16, 1, 9, 2, 5),
     ("bf16", 64, 8, 4, 33, 1, 0),
+    # tensor-core prefill (head_dim 128, 128-row tiles in pairs): GQA group 1 (70 tokens, one
+    # partial tile), 2 (150 tokens: three 64-token tiles, the second pair's second tile empty,
+    # local blocks two whole and one ragged), 8 (33 tokens: three 16-token tiles); each then a
+    # second multi-token call over the filled cache
+    ("bf16", 128, 8, 8, 70, 5, 3),
+    ("bf16", 128, 16, 8, 150, 3, 4),
+    ("bf16", 128, 64, 8, 33, 31, 2),
     # one-token decode kernel (head_dim 128, GQA group 2..16), with and without memory rows
     ("bf16", 128, 16, 8, 20, 1, 3),
     ("bf16", 128, 64, 8, 11, 1, 2),

@@ -310,9 +310,12 @@ msa_status launch_topk(const msa_memory *mem, const float *state, const uint8_t 
   return MSA_OK;
 }
 
+// q_early: Qr is the caller's (written by no kernel of this library), so the query
+// normalisation may read it before the previous kernel completes.
 msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, int B, int T, int k,
                       const uint8_t *exclude, float *state, int32_t *ids, float *scores,
-                      void *ws, size_t ws_bytes, cudaStream_t st, int q_pitch = 0) {
+                      void *ws, size_t ws_bytes, cudaStream_t st, int q_pitch = 0,
+                      bool q_early = false) {
   if (q_pitch <= 0) q_pitch = T;
   if (!mem) return fail(MSA_ERR_INVALID_ARG, "null memory");
   if (B < 1 || T < 0) return fail(MSA_ERR_INVALID_ARG, "batch must be >= 1 and tokens >= 0");
@@ -339,7 +342,8 @@ msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, i
     if (mem->dtype == MSA_BF16) {
       auto *qh = reinterpret_cast<__nv_bfloat16 *>(wsb + plan.qhat);
       MSA_CUDA(launch_pdl(msa::qnorm_kernel<__nv_bfloat16>, dim3(R), dim3(thr), 0, st,
-                          static_cast<const __nv_bfloat16 *>(Qr), W, mem->d_r, T, q_pitch, qh));
+                          static_cast<const __nv_bfloat16 *>(Qr), W, mem->d_r, T, q_pitch, qh,
+                          q_early ? 1 : 0));
       MSA_LAUNCHED("qnorm_kernel");
       msa_status s;
       if (R <= 16)
@@ -356,7 +360,7 @@ msa_status route_impl(const msa_memory *mem, const void *keys, const void *Qr, i
     } else {
       auto *qh = reinterpret_cast<float *>(wsb + plan.qhat);
       msa::qnorm_kernel<float><<<R, thr, 0, st>>>(static_cast<const float *>(Qr), W, mem->d_r, T,
-                                                  q_pitch, qh);
+                                                  q_pitch, qh, 0);
       MSA_LAUNCHED("qnorm_kernel");
       dim3 grid(static_cast<unsigned>((mem->n_chunks + 31) / 32), static_cast<unsigned>((R + 31) / 32));
       if (grid.y > 65535) return fail(MSA_ERR_UNSUPPORTED, "too many query rows for fp32 route");
@@ -820,7 +824,7 @@ msa_status msa_route(const msa_memory *mem, const void *router_keys, const void 
                      int32_t tokens, int32_t k, const uint8_t *exclude, float *state, int32_t *ids,
                      float *scores, void *workspace, size_t workspace_bytes, msa_stream stream) {
   return route_impl(mem, router_keys, Qr, batch, tokens, k, exclude, state, ids, scores, workspace,
-                    workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+                    workspace_bytes, reinterpret_cast<cudaStream_t>(stream), 0, true);
 }
 
 size_t msa_attend_workspace_size(const msa_memory *mem, int32_t batch, int32_t tokens, int32_t k,
@@ -880,7 +884,7 @@ msa_status msa_step(const msa_memory *mem, const void *router_keys, const void *
   const size_t route_bytes = round256(plan_route(mem, s->batch, 1, s->top_k).bytes);
   uint8_t *ws = static_cast<uint8_t *>(s->workspace);
   msa_status r = route_impl(mem, router_keys, Qr_tok, s->batch, 1, s->top_k, nullptr, s->state,
-                            s->ids, s->scores, ws, route_bytes, st);
+                            s->ids, s->scores, ws, route_bytes, st, 0, true);
   if (r != MSA_OK) return r;
   // the kernel before the attention is the route's top-k, which writes none of cache_len, the
   // token's Q/K/V or the local cache: the attention may start on its local part early
@@ -1054,7 +1058,7 @@ msa_status msa_step_host(const msa_memory *mem, const void *router_keys, msa_fet
   const size_t route_bytes = round256(plan_route(mem, s->batch, 1, s->top_k).bytes);
   uint8_t *ws = static_cast<uint8_t *>(s->workspace);
   msa_status r = route_impl(mem, router_keys, Qr_tok, s->batch, 1, s->top_k, nullptr, s->state,
-                            s->ids, s->scores, ws, route_bytes, st);
+                            s->ids, s->scores, ws, route_bytes, st, 0, true);
   if (r != MSA_OK) return r;
   r = msa_fetch(f, s->ids, s->batch, s->top_k, stream, fetch_stream);
   if (r != MSA_OK) return r;
@@ -1133,7 +1137,7 @@ static msa_status interleave_impl(const msa_memory *mem, const void *router_keys
       MSA_LAUNCHED("hold_state_kernel");
     }
     r = route_impl(mem, router_keys, q, batch, T, k, taken, state, ids_r, sc_r, ws, plan.rows, st,
-                   q == Qr ? T : plan.cap);
+                   q == Qr ? T : plan.cap, q == Qr);
     if (r != MSA_OK) return r;
     if (hold) {
       msa::hold_state_kernel<<<batch, 256, 0, st>>>(state, saved, count, mem->n_docs, 1);

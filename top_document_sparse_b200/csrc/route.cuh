@@ -19,12 +19,17 @@ namespace msa {
 // Row r = b * T + t of the output reads input row b * pitch + t.
 // The route kernel that follows may start at once: before its own wait it
 // only loads router keys, which no kernel of this library that releases its
-// dependents early ever writes.
+// dependents early ever writes.  With `early` (the query rows are the
+// caller's, which no kernel of this library writes) the rows are normalised
+// while the previous kernel still runs, and the wait for it comes last, so
+// that this kernel still completes after it; Q_hat was last read by the
+// previous route's MMAs, which completed before that route released its
+// dependents.
 template <typename T>
 __global__ void qnorm_kernel(const T *__restrict__ Qr, int W, int d_r, int T_tok, int pitch,
-                             T *__restrict__ out) {
+                             T *__restrict__ out, int early) {
   griddep_launch();
-  griddep_wait();
+  if (!early) griddep_wait();
   const int64_t r = blockIdx.x;
   const int64_t src_row = (r / T_tok) * pitch + r % T_tok;
   const int e0 = threadIdx.x * 4;
@@ -39,6 +44,7 @@ __global__ void qnorm_kernel(const T *__restrict__ Qr, int W, int d_r, int T_tok
 #pragma unroll
   for (int e = 0; e < 4; ++e) v[e] *= inv;
   if (active) store4(out + r * W + e0, v);
+  if (early) griddep_wait();
 }
 
 // ---------------------------------------------------------------- epilogue
