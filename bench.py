@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-100m", action="store_true", help="skip the 100M-token host-tier run")
     ap.add_argument("--no-interleave", action="store_true", help="skip the Memory Interleave run")
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip the merge / update / backward timings")
     return ap.parse_args()
 
 
@@ -987,6 +989,12 @@ def main():
         from top_document_sparse_b200 import msa
         torch.cuda.empty_cache()
         res["interleave"] = run_interleave(WORKLOADS["interleave_bf16"], msa)
+    if not args.no_next and world == 1 and w.name == "mem1m_bf16":
+        # the widening calls at the same memory: Memory Parallel's merge of four shards'
+        # candidates, the incremental update of one document, the backward of one decode token
+        from top_document_sparse_b200 import kernel_bench
+        torch.cuda.empty_cache()
+        res["next_rows"] = kernel_bench.run(w.name, ["merge", "update", "backward"], reps=3)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
