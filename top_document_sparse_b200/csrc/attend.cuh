@@ -219,10 +219,12 @@ attend_simt_kernel(const T *__restrict__ content, const int32_t *__restrict__ id
 // CTAs share an SM, so the 8 x 64 (query, kv head) CTAs of a decode batch run in one wave.
 constexpr int kAttWarps = 3;
 constexpr int kAttRows = 16;  // context rows per warp block
-// Early path: local blocks past the ring's first that a warp prefetches into L2
-// while the previous kernel (the top-k, which leaves HBM idle) finishes.
+// Early path: local blocks past the ring's first that a warp may prefetch into
+// L2 while the previous kernel (the top-k) finishes.  None by default: measured
+// on the 1M decode once the query normalisation ran before its dependency wait,
+// 1,543 steps/s with none, 1,494 with two blocks, 1,475 with four.
 #ifndef MSA_ATT_EARLY_L2
-#define MSA_ATT_EARLY_L2 2
+#define MSA_ATT_EARLY_L2 0
 #endif
 constexpr int kAttEarlyL2 = MSA_ATT_EARLY_L2;
 
