@@ -84,6 +84,21 @@ def test_full_size_route_and_decode_on_sampled_outputs(name):
     else:
         mem.sparse_attend(ct, layer.ids, Q, Kn, Vn, layer.k_cache, layer.v_cache, layer.cache_len,
                           k, O, ws_a)
+    # the prefill attention (the tensor-core kernel) of the sampled queries, every token, over
+    # the documents the prefill route retrieved
+    torch.cuda.synchronize()
+    assert msa.device_error() == 0
+    ids_pre = layer.ids.cpu().numpy()
+    for b in q_sample:
+        docs = [int(d) for d in ids_pre[b]]
+        enc = [_oracle_doc(keep, d, w) for d in docs]
+        Kb = np.concatenate([e[0] for e in enc])
+        Vb = np.concatenate([e[1] for e in enc])
+        mini_off = np.concatenate([[0], np.cumsum([e[0].shape[0] for e in enc])])
+        ref, _, _ = oracle.attend(Q[b:b + 1].cpu(), Kn[b:b + 1].cpu(), Vn[b:b + 1].cpu(), 0, Kb, Vb,
+                                  mini_off, np.arange(len(docs), dtype=np.int32)[None], k,
+                                  w.rope_theta)
+        assert_close(O[b:b + 1], ref, 1e-2 + 0.5 * bf16_ulp(ref), f"prefill attention of query {b}")
     # every decode position of the workload, checked at four of them (first, two middle, last)
     S = w.decode_steps
     checks = sorted({0, S // 3, (2 * S) // 3, S - 1})
