@@ -217,3 +217,23 @@ def test_full_size_interleave_on_sampled_queries():
             rows = np.concatenate([Krb[cho[d]:cho[d + 1]] for d in g], axis=0)
     print(f"interleave: {len(missed)} of {B} queries missed a hop; sampled {sample}; "
           f"the missed hops against the oracle's k-th score: {miss_kinds}")
+    # the sparse generation step over the R * k retrieved documents, launched as the bench
+    # launches it (a multi-token call on the tensor-core kernel), checked stage-wise on the
+    # GPU's stored pooled rows for two sampled queries, every token
+    _, Qa, Kna, Vna = inputs.queries(w, B, T, seed + 1, "cuda")
+    ctx_ids = ids.permute(1, 0, 2).reshape(B, R * k).contiguous()
+    Kc = torch.zeros(B, T, w.n_kv_heads, w.head_dim, dtype=torch.bfloat16, device="cuda")
+    Vc = torch.zeros_like(Kc)
+    clen = torch.zeros(B, dtype=torch.int32, device="cuda")
+    O = torch.empty(B, T, w.n_q_heads, w.head_dim, dtype=torch.bfloat16, device="cuda")
+    mem.sparse_attend(ct, ctx_ids, Qa, Kna, Vna, Kc, Vc, clen, R * k, O,
+                      msa.workspace(mem.attend_workspace_size(B, T, R * k, w.n_q_heads)))
+    torch.cuda.synchronize()
+    assert msa.device_error() == 0
+    Kb, Vb = to64(ct[:, 0]), to64(ct[:, 1])
+    for q in sample[:2]:
+        docs = ctx_ids[q].cpu().numpy().astype(np.int32)
+        ref, _, _ = oracle.attend(Qa[q:q + 1].cpu(), Kna[q:q + 1].cpu(), Vna[q:q + 1].cpu(), 0, Kb,
+                                  Vb, cho, docs[None], R * k, w.rope_theta)
+        assert_close(O[q:q + 1], ref, 1e-2 + 0.5 * bf16_ulp(ref),
+                     f"final attention of query {q} over {R * k} documents")
